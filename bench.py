@@ -1,0 +1,388 @@
+#!/usr/bin/env python
+"""Throughput of the biased-attention forward on B200: TFLOP/s and % of roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload tri_1024] [--impl ours|reference]
+
+A step is one evo_attn_fwd call over one batch of the workload (default: the
+large triangle-attention case, B=1, N=S=1024, H=4, D=32, bf16, synthetic
+seeded inputs).  FLOPs per step are 4*B*N*H*S^2*D.  The kernel-only number
+(``value``) times K back-to-back calls on inputs resident in HBM (1.1 GB of
+inputs, larger than the 126 MB L2, so no flush is needed between steps) with
+CUDA events on the launching stream, bracketed by a barrier and a device
+synchronize, max over ranks.  ``e2e`` times the same call with the inputs
+copied from pinned host memory and O / LSE copied back inside every step.
+
+Multi-GPU: the forward pass has no exchange step; each rank runs its own
+replica of the workload on its own GPU (weak scaling, no data-path
+collective).  ``--impl reference`` times the float64 CPU oracle instead (rank
+0 only), on a bounded sample of (b, n, h) slices per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from triangle_biased_attention_b200 import workloads as W  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+KERNEL_SOURCES = ["common.cuh", "ptx_sm100.cuh", "fwd_bf16_sm100.cuh", "evo_attn.cu"]
+KERNEL_NAME = "evo_fwd_bf16_kernel"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="tri_1024", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ plumbing
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if (args.impl == "ours" and torch.cuda.is_available()) else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"]))}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "triangle_biased_attention_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[workload]
+        if e.get("kernel_source_hash") == kernel_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        pass
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML unavailable: no clock record
+            self._nv = None
+        self.period = period_s
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def record(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ oracle leg
+def time_oracle(case, slices_per_step: int, steps: int, warmup: int, seed: int):
+    """Times the float64 CPU oracle on `steps` samples of `slices_per_step`
+    (b, n, h) slices each.  Returns (seconds per step, flops per step, cores)."""
+    import oracle
+    B, N, S, H, D = case.shape
+    total = B * N * H
+    rng = torch.Generator().manual_seed(seed)
+    cores = oracle.max_threads()
+    flops_slice = 4 * S * S * D
+    per_step = []
+
+    def sample():
+        idx = torch.randint(0, total, (slices_per_step,), generator=rng).tolist()
+        return [(i // (N * H), (i // H) % N, i % H) for i in idx]
+
+    for _ in range(warmup):
+        oracle.attention_slices(case.q, case.k, case.v, case.mask, case.pair, sample())
+    for _ in range(steps):
+        sl = sample()
+        t0 = time.perf_counter()
+        oracle.attention_slices(case.q, case.k, case.v, case.mask, case.pair, sl)
+        per_step.append(time.perf_counter() - t0)
+    return sum(per_step) / len(per_step), flops_slice * slices_per_step, cores
+
+
+def cpu_baseline(case, args, target_s: float = 10.0):
+    """The oracle on random (b, n, h) slices of the workload, in chunks of
+    4 slices per host core, until about `target_s` seconds have been spent."""
+    import oracle
+    cores = oracle.max_threads()
+    chunk = 4 * cores
+    done_sec = done_flops = 0.0
+    n_slices = 0
+    seed = args.seed
+    while done_sec < target_s and n_slices < case.q.shape[0] * case.q.shape[1] * case.q.shape[3]:
+        sec, fl, cores = time_oracle(case, chunk, 1, 0, seed)
+        done_sec += sec
+        done_flops += fl
+        n_slices += chunk
+        seed += 1
+    return {"value": done_flops / done_sec / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n_slices} random (b,n,h) slices of {args.workload} ({done_flops / 1e9:.0f} GFLOP "
+                      f"in {done_sec:.1f} s, float64 C, OpenMP)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    wl = W.WORKLOADS[args.workload]
+    case = W.make_case(args.workload, args.seed)
+    import oracle
+    cores = oracle.max_threads()
+    # each step: one slice per host core, so a step is ~0.1-0.5 s of work
+    slices = max(1, cores)
+    sec, flops, cores = time_oracle(case, slices, args.steps, args.warmup, args.seed)
+    tflops = flops / sec / 1e12
+    line = {
+        "metric": "Evoformer attn fwd TFLOP/s and % of roofline (triangle attn, N_res=1024)",
+        "value": tflops, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64)",
+        "config": workload_config(wl), "impl": "reference",
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{slices} random (b,n,h) slices of {args.workload} per step"},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl):
+    return {"workload": wl.name, "B": wl.B, "N": wl.N, "S": wl.S, "H": wl.H, "D": wl.D,
+            "dtype": "bf16" if wl.dtype == torch.bfloat16 else "fp32",
+            "l2": "inputs (%.2f GB) larger than the 126 MB L2; no flush" % (alg_bytes(wl) / 1e9),
+            "parallelism": "replicas (one full workload per GPU)"}
+
+
+def alg_bytes(wl) -> int:
+    es = 2 if wl.dtype == torch.bfloat16 else 4
+    qkvo = 4 * wl.B * wl.N * wl.S * wl.H * wl.D * es
+    pair = wl.B * wl.H * wl.S * wl.S * es if wl.name != "msa_col_2048" else 0
+    mask = wl.B * wl.N * wl.S * es
+    lse = wl.B * wl.N * wl.H * wl.S * 4
+    return qkvo + pair + mask + lse
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local):
+    import triangle_biased_attention_b200 as evo
+    wl = W.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    case = W.make_case(args.workload, args.seed + rank)
+    q, k, v = (t.to(dev) for t in (case.q, case.k, case.v))
+    mask = case.mask.to(dev) if case.mask is not None else None
+    pair = case.pair.to(dev) if case.pair is not None else None
+    out = torch.empty_like(q)
+    lse = torch.empty((wl.B, wl.N, wl.H, wl.S), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    flops = wl.flops
+
+    def step():
+        evo.evo_attn(q, k, v, mask, pair, out=out, lse=lse, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    status = evo.evo_attn_sync_status(stream.cuda_stream)
+    if status != evo.EVO_OK:
+        raise RuntimeError(f"kernel status {status}: {evo.evo_attn_strerror(status)}")
+
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with sampler:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = start.elapsed_time(stop)
+    status = evo.evo_attn_sync_status(stream.cuda_stream)
+    if status != evo.EVO_OK:
+        raise RuntimeError(f"kernel status {status}: {evo.evo_attn_strerror(status)}")
+    ms_max = max_over_ranks(ms, world, dev)
+    ms_per_step = ms_max / args.steps
+    value = world * flops * args.steps / (ms_max * 1e-3) / 1e12
+
+    # end to end: pinned host inputs -> device -> kernel -> O, LSE back to pinned host
+    host_in = [t.pin_memory() for t in (case.q, case.k, case.v, case.mask, case.pair) if t is not None]
+    dev_in = [q, k, v] + ([mask] if mask is not None else []) + ([pair] if pair is not None else [])
+    host_o = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    host_lse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_o.numel() * host_o.element_size() + host_lse.numel() * host_lse.element_size()
+
+    def e2e_step():
+        for h, d in zip(host_in, dev_in):
+            d.copy_(h, non_blocking=True)
+        o_, l_ = evo.evo_attn(q, k, v, mask, pair, out=out, lse=lse, stream=stream)
+        host_o.copy_(o_, non_blocking=True)
+        host_lse.copy_(l_, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.e2e_steps
+    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms / args.steps * 1e-3) / 1e12  # this rank's kernel, per launch
+    t_flop = flops / (peaks["bf16_tflops"] * 1e12)
+    t_mem = alg_bytes(wl) / (peaks["hbm_gbs"] * 1e9)
+    bound = "tensor" if t_flop >= t_mem else "hbm"
+    if bound == "tensor":
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"]}
+    else:
+        gbs = alg_bytes(wl) / (ms / args.steps * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"]}
+    roof["traffic"] = recorded_traffic(args.workload)
+    roof["peak_source"] = f"{peak_src} (MEASURED_PEAKS.json burst figure)" if peak_src == "measured" \
+        else "fallback (6.65 TB/s, 1.59 PFLOP/s)"
+    roof["alg_flops_per_launch"] = flops
+    roof["alg_bytes_per_launch"] = alg_bytes(wl)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(case, args)
+
+    if rank == 0:
+        line = {
+            "metric": "Evoformer attn fwd TFLOP/s and % of roofline (triangle attn, N_res=1024)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded numpy PCG64, bf16)",
+            "config": workload_config(wl),
+            "roofline_pct": 100.0 * roof["frac"] if bound == "tensor" else 100.0 * roof["frac"],
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms, "steps": args.e2e_steps},
+            "gpu_launches": args.steps,
+            "kernel": KERNEL_NAME,
+            "clocks": sampler.record(),
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,129 @@
+/*
+ * evo_attn.h — C ABI of the B200 (sm_100a) biased-attention forward library,
+ * libevoattn.so.
+ *
+ * The operation is the forward pass that the DeepSpeed DS4Sci_EvoformerAttention
+ * guide (hmyw.cn) describes for the four Evoformer attention variants (its
+ * section 5.3: MSA row-wise, MSA column-wise, triangle attention around the
+ * starting node and around the ending node):
+ *
+ *     O[b,n,i,h,:] = sum_j softmax_j(t)[j] * V[b,n,j,h,:]
+ *     t_j          = Q[b,n,i,h,:] . K[b,n,j,h,:] / sqrt(D)
+ *                    + mask_bias[b,n,0,0,j] + pair_bias[b,0,h,i,j]
+ *     LSE[b,n,h,i] = log sum_j exp(t_j)              (natural log)
+ *
+ * with the unified layout [*, L, Head, Dim] of its section 5.2 written out as
+ * Q, K, V, O = [B, N, S, H, D], the residue-mask bias [B, N, 1, 1, S] and the
+ * pair bias [B, 1, H, S, S] that is shared by every n (section 5.2), and the
+ * FlashAttention-style log-sum-exp the forward kernel also returns (section
+ * 5.4).  The four variants differ only in what N and S mean and in whether a
+ * pair bias is passed (section 5.3); the caller lays the tensors out for the
+ * variant it wants (for the ending-node case it passes the edges of the other
+ * side, already transposed).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    keeps no reference to them after the call returns and allocates nothing
+ *    per call.
+ *  - Tensors are dense and contiguous (row-major in the shapes above).
+ *  - Calls are asynchronous on `stream` (NULL = the legacy default stream);
+ *    the library never synchronises on its own.
+ *  - Arguments are checked before anything is launched; a bad argument
+ *    returns a negative evo_status_t and launches nothing.  The library never
+ *    aborts or throws.
+ *  - A kernel that stops waiting on an internal barrier after about two
+ *    seconds records EVO_ERR_TIMEOUT in a device status word and exits; read
+ *    it with evo_attn_sync_status().
+ */
+#ifndef EVO_ATTN_H
+#define EVO_ATTN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define EVO_API __attribute__((visibility("default")))
+#else
+#define EVO_API
+#endif
+
+/* Same object as cudaStream_t, declared here so that including this header
+ * does not require the CUDA headers. */
+typedef struct CUstream_st* evo_stream_t;
+
+typedef enum {
+    EVO_DTYPE_BF16 = 0,   /* bf16 inputs and O, fp32 arithmetic, tensor cores */
+    EVO_DTYPE_FP32 = 1    /* fp32 inputs and O, fp32 arithmetic throughout    */
+} evo_dtype_t;
+
+typedef enum {
+    EVO_OK                    =  0,
+    EVO_ERR_INVALID_ARG       = -1,  /* NULL pointer, negative size, overlap   */
+    EVO_ERR_UNSUPPORTED_DTYPE = -2,  /* dtype not one of evo_dtype_t           */
+    EVO_ERR_UNSUPPORTED_SHAPE = -3,  /* outside the supported envelope below   */
+    EVO_ERR_MISALIGNED        = -4,  /* a pointer breaks the alignment rule    */
+    EVO_ERR_CUDA              = -5,  /* a CUDA runtime/driver call failed      */
+    EVO_ERR_TIMEOUT           = -6   /* a device-side wait gave up (see above) */
+} evo_status_t;
+
+/*
+ * evo_attn_fwd — the fused forward pass.
+ *
+ *   Q, K, V    [B, N, S, H, D] of `dtype`.
+ *   mask_bias  [B, N, 1, 1, S] of `dtype`, or NULL for no mask bias.  The
+ *              guide's tests pass it as 1e9 * (mask - 1) (section 5.2), so a
+ *              masked key carries -1e9 (-998244352 once rounded to bf16).  A
+ *              row whose every key is masked that way still follows the
+ *              formula: the mask is then a constant shift of the row.  A row
+ *              with no finite logit at all (every key -inf) returns O = 0 and
+ *              LSE = -inf.
+ *   pair_bias  [B, 1, H, S, S] of `dtype`, indexed [.., query i, key j], or
+ *              NULL (the column-wise variant passes none, section 5.3(b)).
+ *   O          [B, N, S, H, D] of `dtype`, written.
+ *   LSE        [B, N, H, S] fp32, natural log, written.  (The guide's kernel
+ *              pads the last axis to a multiple of 32; this one does not.)
+ *   B, N, S, H >= 0 (a zero size is a no-op that returns EVO_OK and may come
+ *              with NULL pointers), D >= 1.
+ *   dtype      an evo_dtype_t.
+ *   stream     CUDA stream the kernel is launched on.
+ *
+ * Supported envelope:
+ *   EVO_DTYPE_BF16: D in {16, 32, 64}; Q, K, V, O, pair_bias 16-byte aligned;
+ *                   with a pair bias, S a multiple of 8 (its rows are read by
+ *                   the tensor-memory accelerator, which needs 16-byte row
+ *                   strides); mask_bias 2-byte aligned.  Runs on tcgen05
+ *                   tensor cores with fp32 accumulation in tensor memory.
+ *   EVO_DTYPE_FP32: 1 <= D <= 128, any S; 4-byte alignment.  Plain fp32 FMA.
+ *   Every element count must fit in int64 and the grid in CUDA's limits.
+ *   O and LSE must not overlap each other or any input.
+ *
+ * Returns EVO_OK once the work is enqueued, or a negative evo_status_t.
+ */
+EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
+                 const void* mask_bias, const void* pair_bias,
+                 void* O, float* LSE,
+                 int64_t B, int64_t N, int64_t S, int64_t H, int64_t D,
+                 int dtype, evo_stream_t stream);
+
+/*
+ * evo_attn_sync_status — synchronise `stream`, then return and clear the
+ * device status word of the current device: EVO_OK, EVO_ERR_TIMEOUT if a
+ * kernel gave up waiting since the last call, or EVO_ERR_CUDA if the stream
+ * itself reports an error.
+ */
+EVO_API int evo_attn_sync_status(evo_stream_t stream);
+
+/* evo_attn_strerror — a static, human-readable string for a status code. */
+EVO_API const char* evo_attn_strerror(int status);
+
+/* evo_attn_version — library version as major*10000 + minor*100 + patch. */
+EVO_API int evo_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EVO_ATTN_H */

@@ -1,0 +1,119 @@
+"""The C-ABI library loads, exports what include/*.h declares, and rejects bad
+arguments with the documented status codes before touching the GPU."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+import triangle_biased_attention_b200 as evo
+from triangle_biased_attention_b200 import build as evo_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    evo_build.build()
+    return evo.load_library()
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names.update(re.findall(r"EVO_API\s+[\w\s\*]*?\b(evo_\w+)\s*\(", text))
+    return names
+
+
+def test_exports_match_header(lib):
+    declared = declared_symbols()
+    assert {"evo_attn_fwd", "evo_attn_sync_status", "evo_attn_strerror", "evo_attn_version"} <= declared
+    out = subprocess.run(["nm", "-D", "--defined-only", evo.library_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    assert declared <= exported, f"declared but not exported: {declared - exported}"
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def test_strerror_and_version(lib):
+    for code in range(-6, 1):
+        s = evo.evo_attn_strerror(code)
+        assert s and s != "unknown status"
+    assert evo.evo_attn_strerror(-99) == "unknown status"
+    assert evo.evo_attn_version() >= 100
+
+
+def call(Q=0x10000, K=0x20000, V=0x30000, M=None, P=None, O=0x100000, L=0x200000,
+         B=1, N=2, S=64, H=2, D=32, dtype=evo.EVO_DTYPE_BF16):
+    return evo.evo_attn_fwd(Q, K, V, M, P, O, L, B, N, S, H, D, dtype, None)
+
+
+def test_zero_sizes_are_noops(lib):
+    for dims in ({"B": 0}, {"N": 0}, {"S": 0}, {"H": 0}):
+        assert call(Q=None, K=None, V=None, O=None, L=None, **dims) == evo.EVO_OK
+
+
+def test_invalid_arguments(lib):
+    assert call(Q=None) == evo.EVO_ERR_INVALID_ARG
+    assert call(L=None) == evo.EVO_ERR_INVALID_ARG
+    assert call(B=-1) == evo.EVO_ERR_INVALID_ARG
+    assert call(S=-5) == evo.EVO_ERR_INVALID_ARG
+    assert call(dtype=7) == evo.EVO_ERR_UNSUPPORTED_DTYPE
+    assert call(dtype=2) == evo.EVO_ERR_UNSUPPORTED_DTYPE   # fp16 is not offered
+    assert call(D=0) == evo.EVO_ERR_UNSUPPORTED_SHAPE
+
+
+def test_overlapping_outputs_rejected(lib):
+    # O overlaps Q
+    assert call(Q=0x100000, O=0x100000 + 64) == evo.EVO_ERR_INVALID_ARG
+    # LSE inside the mask bias
+    assert call(M=0x400000, L=0x400000) == evo.EVO_ERR_INVALID_ARG
+    # O overlaps LSE
+    assert call(L=0x100000 + 16) == evo.EVO_ERR_INVALID_ARG
+
+
+def test_bf16_envelope(lib):
+    for d in (8, 24, 48, 128, 256):
+        assert call(D=d) == evo.EVO_ERR_UNSUPPORTED_SHAPE
+    # a pair bias needs 16-byte rows: S a multiple of 8
+    assert call(S=60, P=0x800000) == evo.EVO_ERR_UNSUPPORTED_SHAPE
+    assert call(Q=0x10008) == evo.EVO_ERR_MISALIGNED
+    assert call(O=0x100002) == evo.EVO_ERR_MISALIGNED
+    assert call(P=0x800008) == evo.EVO_ERR_MISALIGNED
+    assert call(M=0x900001) == evo.EVO_ERR_MISALIGNED
+    assert call(L=0x200002) == evo.EVO_ERR_MISALIGNED
+    far = dict(Q=1 << 40, K=2 << 40, V=3 << 40, O=4 << 40, L=5 << 40)
+    assert call(B=70000, H=1, **far) == evo.EVO_ERR_UNSUPPORTED_SHAPE   # grid z = B*H > 65535
+
+
+def test_fp32_envelope(lib):
+    f = evo.EVO_DTYPE_FP32
+    assert call(D=129, dtype=f) == evo.EVO_ERR_UNSUPPORTED_SHAPE
+    assert call(Q=0x10002, dtype=f) == evo.EVO_ERR_MISALIGNED
+    assert call(M=0x900002, dtype=f) == evo.EVO_ERR_MISALIGNED
+
+
+def test_size_overflow_rejected(lib):
+    assert call(B=1 << 40, N=1 << 40) == evo.EVO_ERR_UNSUPPORTED_SHAPE
+
+
+def test_python_wrapper_validates_before_calling():
+    import torch
+    q = torch.zeros(1, 2, 8, 1, 16)
+    with pytest.raises(ValueError):
+        evo.evo_attn(q, q, q)          # CPU tensors are refused
+    with pytest.raises(ValueError):
+        evo.evo_attn(q, q[:, :1], q)   # shape mismatch
+    with pytest.raises(TypeError):
+        evo.evo_attn(q.double(), q.double(), q.double())
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(evo, "_lib", None)
+    monkeypatch.setattr(evo, "_LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        evo.load_library()

@@ -1,0 +1,147 @@
+"""B200-native biased (Evoformer / Pairformer / triangle) attention forward.
+
+The computation is the forward pass of the DeepSpeed DS4Sci_EvoformerAttention
+guide (hmyw.cn, sections 4, 5.2-5.4):
+
+    O   = softmax(Q K^T / sqrt(D) + mask_bias + pair_bias) V
+    LSE = log sum exp of the same logits (natural log, fp32)
+
+with Q, K, V, O of shape [B, N, S, H, D], mask_bias [B, N, 1, 1, S] and
+pair_bias [B, 1, H, S, S] (shared by every n).  All arithmetic runs in the
+CUDA library ``libevoattn.so`` (hand-written sm_100a kernels behind the C ABI
+in ``include/evo_attn.h``); this module only marshals arguments through
+ctypes.  PyTorch supplies device memory and the current stream.  There is no
+fallback: without the built library every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = [
+    "evo_attn", "evo_attn_fwd", "evo_attn_sync_status", "evo_attn_strerror", "evo_attn_version",
+    "EvoAttnError", "library_path", "load_library",
+    "EVO_DTYPE_BF16", "EVO_DTYPE_FP32",
+    "EVO_OK", "EVO_ERR_INVALID_ARG", "EVO_ERR_UNSUPPORTED_DTYPE", "EVO_ERR_UNSUPPORTED_SHAPE",
+    "EVO_ERR_MISALIGNED", "EVO_ERR_CUDA", "EVO_ERR_TIMEOUT",
+]
+
+EVO_DTYPE_BF16 = 0
+EVO_DTYPE_FP32 = 1
+
+EVO_OK = 0
+EVO_ERR_INVALID_ARG = -1
+EVO_ERR_UNSUPPORTED_DTYPE = -2
+EVO_ERR_UNSUPPORTED_SHAPE = -3
+EVO_ERR_MISALIGNED = -4
+EVO_ERR_CUDA = -5
+EVO_ERR_TIMEOUT = -6
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libevoattn.so")
+_lib = None
+
+_DTYPES = {torch.bfloat16: EVO_DTYPE_BF16, torch.float32: EVO_DTYPE_FP32}
+
+
+class EvoAttnError(RuntimeError):
+    def __init__(self, status: int, what: str = "evo_attn_fwd"):
+        self.status = status
+        super().__init__(f"{what} failed with status {status}: {evo_attn_strerror(status)}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libevoattn.so (built in-tree by ``build.py``); raise if it is absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(
+            f"{_LIB_PATH} is missing: build it with `python -m triangle_biased_attention_b200.build` "
+            "(there is no fallback implementation)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.evo_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, vp]
+    lib.evo_attn_fwd.restype = i32
+    lib.evo_attn_sync_status.argtypes = [vp]
+    lib.evo_attn_sync_status.restype = i32
+    lib.evo_attn_strerror.argtypes = [i32]
+    lib.evo_attn_strerror.restype = ctypes.c_char_p
+    lib.evo_attn_version.argtypes = []
+    lib.evo_attn_version.restype = i32
+    _lib = lib
+    return lib
+
+
+def evo_attn_fwd(Q: int, K: int, V: int, mask_bias: Optional[int], pair_bias: Optional[int], O: int, LSE: int,
+                 B: int, N: int, S: int, H: int, D: int, dtype: int, stream: Optional[int]) -> int:
+    """The C entry point with raw addresses (ints); returns the status code."""
+    return int(load_library().evo_attn_fwd(Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, dtype, stream))
+
+
+def evo_attn_sync_status(stream: Optional[int] = None) -> int:
+    return int(load_library().evo_attn_sync_status(stream))
+
+
+def evo_attn_strerror(status: int) -> str:
+    return load_library().evo_attn_strerror(int(status)).decode()
+
+
+def evo_attn_version() -> int:
+    return int(load_library().evo_attn_version())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def evo_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+             mask: Optional[torch.Tensor] = None, pair: Optional[torch.Tensor] = None,
+             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+             stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Biased-attention forward on CUDA tensors; returns (O, LSE).
+
+    q, k, v: [B, N, S, H, D] bf16 or fp32, contiguous, on one CUDA device.
+    mask: [B, N, 1, 1, S] or None.  pair: [B, 1, H, S, S] or None (same dtype).
+    out / lse: optional preallocated outputs ([B, N, S, H, D], [B, N, H, S] fp32).
+    Runs on ``stream`` (default: the current stream) without synchronising.
+    """
+    if q.dim() != 5:
+        raise ValueError("q must be [B, N, S, H, D]")
+    B, N, S, H, D = q.shape
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    for name, t, shape in (("k", k, q.shape), ("v", v, q.shape),
+                           ("mask", mask, (B, N, 1, 1, S)), ("pair", pair, (B, 1, H, S, S))):
+        if t is None:
+            continue
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} differs from q dtype {q.dtype}")
+        if t.device != q.device:
+            raise ValueError(f"{name} is on {t.device}, q on {q.device}")
+    for name, t in (("q", q), ("k", k), ("v", v), ("mask", mask), ("pair", pair)):
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if q.device.type != "cuda":
+        raise ValueError("tensors must be on a CUDA device")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, N, H, S), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    status = evo_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(mask), _ptr(pair),
+                          out.data_ptr(), lse.data_ptr(), B, N, S, H, D, _DTYPES[q.dtype],
+                          stream.cuda_stream)
+    if status != EVO_OK:
+        raise EvoAttnError(status)
+    return out, lse

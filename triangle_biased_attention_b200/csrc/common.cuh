@@ -1,0 +1,47 @@
+// Shared device-side plumbing: the library's status word and bounded waits.
+#pragma once
+
+#include <cstdint>
+
+#include "evo_attn.h"
+#include "ptx_sm100.cuh"
+
+namespace evo {
+
+// Device status word of this library (one per device that loads it).  A
+// kernel that gives up waiting records EVO_ERR_TIMEOUT here; the host reads
+// and clears it in evo_attn_sync_status().
+__device__ int g_status;
+
+// A wait on an internal barrier longer than this is treated as a hang.
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+
+__device__ __forceinline__ void record_status(int code) { atomicCAS(&g_status, 0, code); }
+
+// Waits for the given phase parity of an mbarrier.  Returns false, after
+// raising the CTA's abort flag and recording EVO_ERR_TIMEOUT, if the phase
+// does not complete within kWaitTimeoutNs; returns false at once if another
+// thread of the CTA has already raised the flag (pass abort_flag = nullptr to
+// wait regardless of it, as the drain paths do).
+__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (true) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (abort_flag != nullptr && *abort_flag) return false;
+        if (ptx::globaltimer_ns() - t0 > kWaitTimeoutNs) {
+            if (abort_flag != nullptr) *abort_flag = 1;
+            record_status(EVO_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Warp-uniform form: every lane waits (so every lane acquires the barrier),
+// and the warp agrees on the outcome.
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    const bool ok = wait_bounded(bar, parity, abort_flag);
+    return __all_sync(0xffffffffu, ok);
+}
+
+}  // namespace evo

@@ -1,0 +1,270 @@
+// Host side of libevoattn.so: argument checks, TMA tensor-map encoding and
+// kernel launch for the C ABI declared in include/evo_attn.h.
+//
+// The calling convention follows the DeepSpeed DS4Sci_EvoformerAttention
+// guide's statement of the problem (hmyw.cn, section 5: one call for all four
+// variants, Q/K/V in [*, L, Head, Dim], biases [B,N,1,1,S] and [B,1,H,S,S],
+// a missing bias passed as "empty" -- here NULL -- through the same call, an
+// fp32 log-sum-exp beside O), adapted to plain pointers and status codes: the
+// guide's Python front end asserts on dtype and shapes, this library returns
+// an evo_status_t before launching anything.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "evo_attn.h"
+#include "common.cuh"
+#include "fwd_bf16_sm100.cuh"
+#include "fwd_f32.cuh"
+
+namespace {
+
+using evo::Bf16Cfg;
+
+constexpr int kMaxDevices = 64;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+bool mul_ok(int64_t a, int64_t b, int64_t* out) { return !__builtin_mul_overflow(a, b, out); }
+
+bool overlap(const void* a, int64_t abytes, const void* b, int64_t bbytes) {
+    if (a == nullptr || b == nullptr || abytes <= 0 || bbytes <= 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + uint64_t(bbytes) && b0 < a0 + uint64_t(abytes);
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Make this library's runtime use the device that owns `ptr` (the caller's
+// framework may keep its own notion of the current device).
+int select_device_of(const void* ptr) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, ptr) != cudaSuccess) {
+        cudaGetLastError();
+        return EVO_ERR_INVALID_ARG;
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return EVO_ERR_INVALID_ARG;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return EVO_ERR_CUDA;
+    if (cur != attr.device && cudaSetDevice(attr.device) != cudaSuccess) return EVO_ERR_CUDA;
+    return attr.device;
+}
+
+// Q/K/V/O as a 4-D tensor {D, H, S, B*N}; a box is one (b, n, h) slice's
+// 128 rows of D elements, swizzled over the D*2-byte row.
+bool encode_qkv(CUtensorMap* m, const void* base, int64_t BN, int64_t S, int64_t H, int64_t D) {
+    const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(S), cuuint64_t(BN)};
+    const cuuint64_t strides[3] = {cuuint64_t(D * 2), cuuint64_t(H * D * 2), cuuint64_t(S * H * D * 2)};
+    const cuuint32_t box[4] = {cuuint32_t(D), 1, cuuint32_t(evo::kBM), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                          : (D == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Pair bias as a 3-D tensor {S (key j), S (query i), B*H}; a box is 128
+// queries x 64 keys (128 B rows, 128 B swizzle).
+bool encode_pair(CUtensorMap* m, const void* base, int64_t BH, int64_t S) {
+    const cuuint64_t dims[3] = {cuuint64_t(S), cuuint64_t(S), cuuint64_t(BH)};
+    const cuuint64_t strides[2] = {cuuint64_t(S * 2), cuuint64_t(S * S * 2)};
+    const cuuint32_t box[3] = {64, cuuint32_t(evo::kBM), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, bool HAS_PAIR>
+int launch_bf16(int dev, const void* Q, const void* K, const void* V, const void* mask, const void* pair, void* O,
+                float* LSE, int64_t B, int64_t N, int64_t S, int64_t H, cudaStream_t stream) {
+    using C = Bf16Cfg<D, HAS_PAIR>;
+    auto kernel = evo::evo_fwd_bf16_kernel<D, HAS_PAIR>;
+    static bool attr_set[kMaxDevices] = {};
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+            return EVO_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    CUtensorMap tq, tk, tv, tp;
+    std::memset(&tp, 0, sizeof(tp));
+    if (!encode_qkv(&tq, Q, B * N, S, H, D) || !encode_qkv(&tk, K, B * N, S, H, D) ||
+        !encode_qkv(&tv, V, B * N, S, H, D))
+        return EVO_ERR_CUDA;
+    if (HAS_PAIR && !encode_pair(&tp, pair, B * H, S)) return EVO_ERR_CUDA;
+
+    evo::Bf16Params p;
+    p.mask = static_cast<const uint16_t*>(mask);
+    p.out = static_cast<uint16_t*>(O);
+    p.lse = LSE;
+    p.N = int(N);
+    p.S = int(S);
+    p.H = int(H);
+    p.num_kb = int((S + evo::kBN - 1) / evo::kBN);
+    p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned((N + 1) / 2), unsigned((S + evo::kBM - 1) / evo::kBM), unsigned(B * H));
+    cfg.blockDim = dim3(evo::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    return cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, tp, p) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+}
+
+int launch_f32(int dev, const void* Q, const void* K, const void* V, const void* mask, const void* pair, void* O,
+               float* LSE, int64_t B, int64_t N, int64_t S, int64_t H, int64_t D, cudaStream_t stream) {
+    evo::F32Params p;
+    p.q = static_cast<const float*>(Q);
+    p.k = static_cast<const float*>(K);
+    p.v = static_cast<const float*>(V);
+    p.mask = static_cast<const float*>(mask);
+    p.pair = static_cast<const float*>(pair);
+    p.out = static_cast<float*>(O);
+    p.lse = LSE;
+    p.N = int(N);
+    p.S = int(S);
+    p.H = int(H);
+    p.D = int(D);
+    p.ld = int(D) + 1;
+    p.num_qb = int((S + evo::kF32Rows - 1) / evo::kF32Rows);
+    p.scale = float(1.0 / std::sqrt(double(D)));
+    const size_t smem = sizeof(float) * (size_t(2 * evo::kF32Keys + evo::kF32Rows) * p.ld +
+                                         size_t(evo::kF32Rows) * evo::kF32Keys + evo::kF32Rows);
+    static bool attr_set[kMaxDevices] = {};
+    if (!attr_set[dev]) {
+        const int max_smem = int(sizeof(float) * (size_t(2 * evo::kF32Keys + evo::kF32Rows) * (evo::kF32MaxD + 1) +
+                                                  size_t(evo::kF32Rows) * evo::kF32Keys + evo::kF32Rows));
+        if (cudaFuncSetAttribute(evo::evo_fwd_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) !=
+            cudaSuccess)
+            return EVO_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    const long long blocks = (long long)B * N * H * p.num_qb;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(blocks), 1, 1);
+    cfg.blockDim = dim3(evo::kF32Rows * 32, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, evo::evo_fwd_f32_kernel, p) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V, const void* mask_bias,
+                            const void* pair_bias, void* O, float* LSE, int64_t B, int64_t N, int64_t S, int64_t H,
+                            int64_t D, int dtype, evo_stream_t stream) {
+    if (B < 0 || N < 0 || S < 0 || H < 0 || D < 0) return EVO_ERR_INVALID_ARG;
+    if (dtype != EVO_DTYPE_BF16 && dtype != EVO_DTYPE_FP32) return EVO_ERR_UNSUPPORTED_DTYPE;
+    if (D == 0) return EVO_ERR_UNSUPPORTED_SHAPE;
+    if (B == 0 || N == 0 || S == 0 || H == 0) return EVO_OK;  // nothing to compute
+    if (!Q || !K || !V || !O || !LSE) return EVO_ERR_INVALID_ARG;
+
+    const int64_t es = dtype == EVO_DTYPE_BF16 ? 2 : 4;
+    int64_t bn, bns, bnsh, qkv_elems, qkv_bytes, mask_bytes, bh, pair_elems, pair_bytes, lse_bytes;
+    if (!mul_ok(B, N, &bn) || !mul_ok(bn, S, &bns) || !mul_ok(bns, H, &bnsh) || !mul_ok(bnsh, D, &qkv_elems) ||
+        !mul_ok(qkv_elems, es, &qkv_bytes) || !mul_ok(bns, es, &mask_bytes) || !mul_ok(B, H, &bh) ||
+        !mul_ok(bh, S, &pair_elems) || !mul_ok(pair_elems, S, &pair_elems) ||
+        !mul_ok(pair_elems, es, &pair_bytes) || !mul_ok(bnsh, 4, &lse_bytes))
+        return EVO_ERR_UNSUPPORTED_SHAPE;
+
+    // outputs must not overlap each other or any input
+    const void* ins[5] = {Q, K, V, mask_bias, pair_bias};
+    const int64_t in_bytes[5] = {qkv_bytes, qkv_bytes, qkv_bytes, mask_bytes, pair_bytes};
+    if (overlap(O, qkv_bytes, LSE, lse_bytes)) return EVO_ERR_INVALID_ARG;
+    for (int i = 0; i < 5; ++i)
+        if (overlap(O, qkv_bytes, ins[i], in_bytes[i]) || overlap(LSE, lse_bytes, ins[i], in_bytes[i]))
+            return EVO_ERR_INVALID_ARG;
+
+    if (!aligned(LSE, 4)) return EVO_ERR_MISALIGNED;
+    const int64_t int_max = 2147483647;
+    if (dtype == EVO_DTYPE_BF16) {
+        if (D != 16 && D != 32 && D != 64) return EVO_ERR_UNSUPPORTED_SHAPE;
+        if (pair_bias && (S % 8) != 0) return EVO_ERR_UNSUPPORTED_SHAPE;
+        // TMA coordinates are 32-bit; grid y and z are limited to 65535
+        if (bn > int_max || S > int_max || bh > 65535 || (S + evo::kBM - 1) / evo::kBM > 65535 ||
+            (N + 1) / 2 > int_max || N > int_max || H > int_max)
+            return EVO_ERR_UNSUPPORTED_SHAPE;
+        if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) ||
+            (pair_bias && !aligned(pair_bias, 16)) || (mask_bias && !aligned(mask_bias, 2)))
+            return EVO_ERR_MISALIGNED;
+    } else {
+        if (D > evo::kF32MaxD) return EVO_ERR_UNSUPPORTED_SHAPE;
+        const int64_t num_qb = (S + evo::kF32Rows - 1) / evo::kF32Rows;
+        int64_t blocks;
+        if (!mul_ok(bnsh / S, num_qb, &blocks) || blocks > int_max || S > int_max || N > int_max || H > int_max)
+            return EVO_ERR_UNSUPPORTED_SHAPE;
+        if (!aligned(Q, 4) || !aligned(K, 4) || !aligned(V, 4) || !aligned(O, 4) ||
+            (pair_bias && !aligned(pair_bias, 4)) || (mask_bias && !aligned(mask_bias, 4)))
+            return EVO_ERR_MISALIGNED;
+    }
+
+    const int dev = select_device_of(Q);
+    if (dev < 0) return dev;
+    if (dev >= kMaxDevices) return EVO_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    if (dtype == EVO_DTYPE_FP32) return launch_f32(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, st);
+
+    if (encode_fn() == nullptr) return EVO_ERR_CUDA;
+    const bool has_pair = pair_bias != nullptr;
+#define EVO_LAUNCH(DD)                                                                                \
+    return has_pair ? launch_bf16<DD, true>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st) \
+                    : launch_bf16<DD, false>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st)
+    switch (D) {
+        case 16: EVO_LAUNCH(16);
+        case 32: EVO_LAUNCH(32);
+        default: EVO_LAUNCH(64);
+    }
+#undef EVO_LAUNCH
+}
+
+extern "C" EVO_API int evo_attn_sync_status(evo_stream_t stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return EVO_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, evo::g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return EVO_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return EVO_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbolAsync(evo::g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) !=
+                cudaSuccess ||
+            cudaStreamSynchronize(st) != cudaSuccess)
+            return EVO_ERR_CUDA;
+    }
+    return v;
+}
+
+extern "C" EVO_API const char* evo_attn_strerror(int status) {
+    switch (status) {
+        case EVO_OK: return "ok";
+        case EVO_ERR_INVALID_ARG: return "invalid argument (NULL pointer, negative size or overlapping outputs)";
+        case EVO_ERR_UNSUPPORTED_DTYPE: return "unsupported dtype";
+        case EVO_ERR_UNSUPPORTED_SHAPE: return "shape outside the supported envelope";
+        case EVO_ERR_MISALIGNED: return "a pointer breaks the alignment rule";
+        case EVO_ERR_CUDA: return "a CUDA call failed";
+        case EVO_ERR_TIMEOUT: return "a device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+extern "C" EVO_API int evo_attn_version(void) { return 100; }

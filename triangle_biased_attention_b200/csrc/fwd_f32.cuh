@@ -1,0 +1,149 @@
+// fp32 biased-attention forward: plain FMA arithmetic in fp32 throughout.
+//
+// The same operation as the bf16 kernel (DeepSpeed DS4Sci_EvoformerAttention
+// guide, hmyw.cn, sections 4, 5.2 and 5.4) for fp32 inputs, where tensor-core
+// TF32 would not hold a 1e-5 relative error.  One warp owns one query row;
+// K and V blocks of 64 keys are staged in shared memory for the 8 rows of a
+// CTA.  Each lane scores two keys of a block, the warp takes the block max
+// and sum with xor-shuffles, then each lane accumulates its D/32 output
+// columns.  The mask is rebased per (b, n) by its maximum, as in the bf16
+// kernel, so an n whose every key carries -1e9 still follows the formula.
+#pragma once
+
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace evo {
+
+constexpr int kF32Rows = 8;   // query rows (warps) per CTA
+constexpr int kF32Keys = 64;  // keys per shared-memory block
+constexpr int kF32MaxD = 128;
+
+struct F32Params {
+    const float* q;
+    const float* k;
+    const float* v;
+    const float* mask;  // [B, N, S] or nullptr
+    const float* pair;  // [B, H, S, S] or nullptr
+    float* out;
+    float* lse;
+    int N, S, H, D;
+    int ld;             // padded smem row (D + 1)
+    int num_qb;         // query blocks of kF32Rows per (b, n, h)
+    float scale;        // 1 / sqrt(D)
+};
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__global__ void __launch_bounds__(kF32Rows * 32) evo_fwd_f32_kernel(const F32Params p) {
+    extern __shared__ float fsm[];
+    float* Ks = fsm;                           // [kF32Keys][ld]
+    float* Vs = Ks + kF32Keys * p.ld;          // [kF32Keys][ld]
+    float* Qs = Vs + kF32Keys * p.ld;          // [kF32Rows][ld]
+    float* Ps = Qs + kF32Rows * p.ld;          // [kF32Rows][kF32Keys]
+    float* red = Ps + kF32Rows * kF32Keys;     // [kF32Rows]
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    long long t = blockIdx.x;
+    const int qb = int(t % p.num_qb);
+    t /= p.num_qb;
+    const int h = int(t % p.H);
+    const long long bn = t / p.H;  // b * N + n
+    const long long b = bn / p.N;
+    const int row = qb * kF32Rows + warp;
+    const int D = p.D;
+    const size_t row_stride = size_t(p.H) * D;  // between consecutive s in [B,N,S,H,D]
+    const size_t slice_base = size_t(bn) * p.S * row_stride + size_t(h) * D;
+
+    // per-(b, n) mask rebase
+    const float* mrow = p.mask ? p.mask + size_t(bn) * p.S : nullptr;
+    float c = 0.f;
+    if (mrow) {
+        float mx = -INFINITY;
+        for (int j = threadIdx.x; j < p.S; j += blockDim.x) mx = fmaxf(mx, mrow[j]);
+        mx = warp_max(mx);
+        if (lane == 0) red[warp] = mx;
+        __syncthreads();
+        mx = red[0];
+        for (int i = 1; i < kF32Rows; ++i) mx = fmaxf(mx, red[i]);
+        c = (mx == -INFINITY) ? 0.f : mx;
+    }
+    const float* prow = (p.pair && row < p.S) ? p.pair + (size_t(b) * p.H + h) * size_t(p.S) * p.S + size_t(row) * p.S
+                                               : nullptr;
+
+    for (int d = lane; d < D; d += 32)
+        Qs[warp * p.ld + d] = row < p.S ? p.q[slice_base + size_t(row) * row_stride + d] : 0.f;
+
+    float m = -INFINITY, l = 0.f;
+    float o[kF32MaxD / 32] = {0.f, 0.f, 0.f, 0.f};
+    for (int kb = 0; kb < p.S; kb += kF32Keys) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < kF32Keys * D; i += blockDim.x) {
+            const int jj = i / D, d = i - jj * D;
+            const int key = kb + jj;
+            const size_t off = slice_base + size_t(key) * row_stride + d;
+            Ks[jj * p.ld + d] = key < p.S ? p.k[off] : 0.f;
+            Vs[jj * p.ld + d] = key < p.S ? p.v[off] : 0.f;
+        }
+        __syncthreads();
+        float tj[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int jj = lane + 32 * e;
+            const int key = kb + jj;
+            float x = -INFINITY;
+            if (key < p.S && row < p.S) {
+                float dot = 0.f;
+                for (int d = 0; d < D; ++d) dot = fmaf(Qs[warp * p.ld + d], Ks[jj * p.ld + d], dot);
+                x = dot * p.scale;
+                if (mrow) x += mrow[key] - c;
+                if (prow) x += prow[key];
+            }
+            tj[e] = x;
+        }
+        const float m_new = fmaxf(m, warp_max(fmaxf(tj[0], tj[1])));
+        const float m_safe = (m_new == -INFINITY) ? 0.f : m_new;
+        const float alpha = (m == -INFINITY) ? 0.f : expf(m - m_safe);
+        const float p0 = expf(tj[0] - m_safe);
+        const float p1 = expf(tj[1] - m_safe);
+        l = l * alpha + warp_sum(p0 + p1);
+        Ps[warp * kF32Keys + lane] = p0;
+        Ps[warp * kF32Keys + lane + 32] = p1;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kF32MaxD / 32; ++i) {
+            const int d = lane + 32 * i;
+            if (d < D) {
+                float acc = o[i] * alpha;
+                for (int jj = 0; jj < kF32Keys; ++jj) acc = fmaf(Ps[warp * kF32Keys + jj], Vs[jj * p.ld + d], acc);
+                o[i] = acc;
+            }
+        }
+        m = m_new;
+        __syncwarp();
+    }
+    if (row < p.S) {
+        const float inv_l = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+        for (int i = 0; i < kF32MaxD / 32; ++i) {
+            const int d = lane + 32 * i;
+            if (d < D) p.out[slice_base + size_t(row) * row_stride + d] = o[i] * inv_l;
+        }
+        if (lane == 0)
+            p.lse[(size_t(bn) * p.H + h) * size_t(p.S) + row] = l > 0.f ? m + logf(l) + c : -INFINITY;
+    }
+}
+
+}  // namespace evo
