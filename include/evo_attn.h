@@ -66,7 +66,9 @@ typedef enum {
     EVO_ERR_UNSUPPORTED_SHAPE = -3,  /* outside the supported envelope below   */
     EVO_ERR_MISALIGNED        = -4,  /* a pointer breaks the alignment rule    */
     EVO_ERR_CUDA              = -5,  /* a CUDA runtime/driver call failed      */
-    EVO_ERR_TIMEOUT           = -6   /* a device-side wait gave up (see above) */
+    EVO_ERR_TIMEOUT           = -6,  /* a device-side wait gave up (see above) */
+    EVO_ERR_RANGE             = -7   /* an input value is outside the range the
+                                        kernel's arithmetic supports (see below) */
 } evo_status_t;
 
 /*
@@ -96,6 +98,10 @@ typedef enum {
  *                   the tensor-memory accelerator, which needs 16-byte row
  *                   strides); mask_bias 2-byte aligned.  Runs on tcgen05
  *                   tensor cores with fp32 accumulation in tensor memory.
+ *                   The softmax numerators P are rounded to fp16 for the P.V
+ *                   product, so V is converted to fp16 on chip: every |V|
+ *                   must be <= 65504, else the kernel records EVO_ERR_RANGE
+ *                   (read by evo_attn_sync_status) and O is not valid.
  *   EVO_DTYPE_FP32: 1 <= D <= 128, any S; 4-byte alignment.  Plain fp32 FMA.
  *   Every element count must fit in int64 and the grid in CUDA's limits.
  *   O and LSE must not overlap each other or any input.
@@ -111,8 +117,9 @@ EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
 /*
  * evo_attn_sync_status — synchronise `stream`, then return and clear the
  * device status word of the current device: EVO_OK, EVO_ERR_TIMEOUT if a
- * kernel gave up waiting since the last call, or EVO_ERR_CUDA if the stream
- * itself reports an error.
+ * kernel gave up waiting since the last call, EVO_ERR_RANGE if a kernel met
+ * an out-of-range input, or EVO_ERR_CUDA if the stream itself reports an
+ * error.  The first error recorded since the last call is the one returned.
  */
 EVO_API int evo_attn_sync_status(evo_stream_t stream);
 

@@ -40,7 +40,7 @@ def test_exports_match_header(lib):
 
 
 def test_strerror_and_version(lib):
-    for code in range(-6, 1):
+    for code in range(-7, 1):
         s = evo.evo_attn_strerror(code)
         assert s and s != "unknown status"
     assert evo.evo_attn_strerror(-99) == "unknown status"
@@ -86,8 +86,9 @@ def test_bf16_envelope(lib):
     assert call(P=0x800008) == evo.EVO_ERR_MISALIGNED
     assert call(M=0x900001) == evo.EVO_ERR_MISALIGNED
     assert call(L=0x200002) == evo.EVO_ERR_MISALIGNED
-    far = dict(Q=1 << 40, K=2 << 40, V=3 << 40, O=4 << 40, L=5 << 40)
-    assert call(B=70000, H=1, **far) == evo.EVO_ERR_UNSUPPORTED_SHAPE   # grid z = B*H > 65535
+    far = dict(Q=1 << 50, K=2 << 50, V=3 << 50, O=4 << 50, L=5 << 50)
+    # CTA count = query blocks x heads x n pairs x batch beyond 2^31 - 1
+    assert call(B=1 << 15, N=1 << 10, S=1 << 10, H=1 << 4, D=16, **far) == evo.EVO_ERR_UNSUPPORTED_SHAPE
 
 
 def test_fp32_envelope(lib):

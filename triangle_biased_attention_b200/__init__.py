@@ -26,7 +26,7 @@ __all__ = [
     "EvoAttnError", "library_path", "load_library",
     "EVO_DTYPE_BF16", "EVO_DTYPE_FP32",
     "EVO_OK", "EVO_ERR_INVALID_ARG", "EVO_ERR_UNSUPPORTED_DTYPE", "EVO_ERR_UNSUPPORTED_SHAPE",
-    "EVO_ERR_MISALIGNED", "EVO_ERR_CUDA", "EVO_ERR_TIMEOUT",
+    "EVO_ERR_MISALIGNED", "EVO_ERR_CUDA", "EVO_ERR_TIMEOUT", "EVO_ERR_RANGE",
 ]
 
 EVO_DTYPE_BF16 = 0
@@ -39,6 +39,7 @@ EVO_ERR_UNSUPPORTED_SHAPE = -3
 EVO_ERR_MISALIGNED = -4
 EVO_ERR_CUDA = -5
 EVO_ERR_TIMEOUT = -6
+EVO_ERR_RANGE = -7
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libevoattn.so")

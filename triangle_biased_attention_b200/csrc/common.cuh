@@ -37,10 +37,16 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+// Inline fast path: one try_wait, then the bounded slow path.
+__device__ __forceinline__ bool wait_fast(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    return wait_bounded(bar, parity, abort_flag);
+}
+
 // Warp-uniform form: every lane waits (so every lane acquires the barrier),
 // and the warp agrees on the outcome.
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    const bool ok = wait_bounded(bar, parity, abort_flag);
+    const bool ok = wait_fast(bar, parity, abort_flag);
     return __all_sync(0xffffffffu, ok);
 }
 

@@ -118,10 +118,12 @@ int launch_bf16(int dev, const void* Q, const void* K, const void* V, const void
     p.S = int(S);
     p.H = int(H);
     p.num_kb = int((S + evo::kBN - 1) / evo::kBN);
+    p.num_qb = int((S + evo::kBM - 1) / evo::kBM);
+    p.num_np = int((N + 1) / 2);
     p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned((N + 1) / 2), unsigned((S + evo::kBM - 1) / evo::kBM), unsigned(B * H));
+    cfg.gridDim = dim3(unsigned(int64_t(p.num_qb) * H * p.num_np * B), 1, 1);
     cfg.blockDim = dim3(evo::kThreads, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
@@ -199,9 +201,12 @@ extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
     if (dtype == EVO_DTYPE_BF16) {
         if (D != 16 && D != 32 && D != 64) return EVO_ERR_UNSUPPORTED_SHAPE;
         if (pair_bias && (S % 8) != 0) return EVO_ERR_UNSUPPORTED_SHAPE;
-        // TMA coordinates are 32-bit; grid y and z are limited to 65535
-        if (bn > int_max || S > int_max || bh > 65535 || (S + evo::kBM - 1) / evo::kBM > 65535 ||
-            (N + 1) / 2 > int_max || N > int_max || H > int_max)
+        // TMA coordinates are 32-bit; the CTA count (query blocks x heads x
+        // n pairs x batch) must fit the grid's x dimension
+        int64_t ctas;
+        if (bn > int_max || bh > int_max || S > int_max || N > int_max || H > int_max ||
+            !mul_ok((S + evo::kBM - 1) / evo::kBM, bh, &ctas) || !mul_ok(ctas, (N + 1) / 2, &ctas) ||
+            ctas > int_max)
             return EVO_ERR_UNSUPPORTED_SHAPE;
         if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) ||
             (pair_bias && !aligned(pair_bias, 16)) || (mask_bias && !aligned(mask_bias, 2)))
@@ -263,6 +268,7 @@ extern "C" EVO_API const char* evo_attn_strerror(int status) {
         case EVO_ERR_MISALIGNED: return "a pointer breaks the alignment rule";
         case EVO_ERR_CUDA: return "a CUDA call failed";
         case EVO_ERR_TIMEOUT: return "a device-side wait timed out";
+        case EVO_ERR_RANGE: return "an input value is outside the supported range (|V| > 65504 with bf16)";
         default: return "unknown status";
     }
 }

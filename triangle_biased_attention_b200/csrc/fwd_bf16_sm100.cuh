@@ -10,22 +10,43 @@
 //  * One CTA owns one (b, h, 128-query block) and TWO n slices, n0 and n0+1.
 //    The pair bias [B,1,H,S,S] does not depend on n, so both slices read the
 //    same 128x128 bias tile from shared memory: one L2->SM transfer feeds two
-//    softmax warpgroups.
-//  * Warp roles (384 threads): warp 0 issues TMA loads (Q once; K, V and bias
-//    tiles through rings of mbarrier-tracked stages); warp 1 issues tcgen05
-//    MMAs from one thread; warp 2 turns the mask row into a log2-scaled fp32
-//    vector per key block (and computes the per-(b,n) rebase, below); warps
-//    4-7 and 8-11 are the softmax warpgroups of slice n0 and n0+1.  Thread r of
-//    a warpgroup owns query row r, which is TMEM lane r, so row max and row sum
-//    stay in one thread.
+//    softmax warpgroups.  CTAs are numbered query block fastest, then head,
+//    so the CTAs that share one (n, h) K/V slice, and the four heads that
+//    share each 256 B stretch of a Q/K/V row, run at the same time and hit L2.
+//  * Warp roles (608 threads, 19 warps): warp 0 issues TMA loads (Q once; K,
+//    V and bias tiles through rings of mbarrier-tracked stages); warp 1 issues
+//    tcgen05 MMAs from one thread; warp 2 turns the mask row into a
+//    log2-scaled fp32 vector per key block (with the per-(b,n) rebase below);
+//    warps 3-18 are softmax warps, eight per slice, each owning 16 query rows
+//    (TMEM lanes) through the 16-lane `16x64b` tensor-memory shape: the two
+//    threads of a row hold its even and its odd key columns, so a row maximum
+//    is one shuffle and no barrier couples the softmax warps; they drift apart
+//    and the exp unit of one overlaps the FMA/ALU work of another.  Each
+//    softmax warp also converts 16 rows of its slice's V tile to fp16 before
+//    it reports P ready, so the P.V MMA that waits for P also finds V
+//    converted.
 //  * Tensor memory (512 columns): per slice, S = Q K^T (128 fp32 columns),
-//    P = softmax numerators as bf16 (64 columns) and the O accumulator
-//    (D columns).  S and P are separate so the next block's Q K^T can start as
-//    soon as the softmax has pulled S into registers.
+//    P = softmax numerators as fp16 (64 columns) and the O accumulator.  S and
+//    P are separate so the next block's Q K^T can start as soon as the softmax
+//    has pulled S into registers.
+//  * P is packed from a thread's own (interleaved) columns, so within every
+//    group of four keys the MMA sees key order 0, 2, 1, 3; the V conversion
+//    swaps rows 1 and 2 of every group of four to match (a permutation of
+//    the contraction index leaves P.V unchanged).
+//  * P is rounded to fp16, not bf16: its 11-bit significand keeps the P.V
+//    rounding error eight times below bf16's, which holds |dO| under 1e-2
+//    next to the bf16 rounding of O itself.  MMA operands share one type, so
+//    V is converted to fp16 in shared memory (exact for |V| <= 65504; larger
+//    values are reported as EVO_ERR_RANGE).
+//  * For D <= 32 the row sum comes from the tensor core: each V stage is
+//    followed by a constant tile whose first column is 1.0, and the P.V MMA
+//    runs with N = D + 16, so O's column D accumulates sum_j P_j (the same
+//    rounded P that weights V) and is rescaled together with O.
 //  * Online softmax in base 2: u = s*log2(e)/sqrt(D) + (pair + mask - c)*log2(e),
-//    p = 2^(u - m).  The running maximum m is only moved when the block maximum
-//    exceeds it by more than 8 (p <= 256, exact after the final division by
-//    the row sum); moving it rescales O in tensor memory.
+//    p = 2^(u - m), with packed f32x2 FMA/ADD.  The running maximum m is only
+//    moved when the block maximum exceeds it by more than 8 (p <= 256, exact
+//    after the final division by the row sum); moving it rescales O in
+//    tensor memory.
 //  * Mask rebase: c[b,n] = max_j mask[b,n,j] is subtracted from the mask and
 //    added back to the LSE.  The guide builds masks as 1e9*(mask-1) (section
 //    5.2); for an n whose every key is masked that is a constant shift of the
@@ -50,12 +71,15 @@ struct Bf16Params {
     float* lse;            // [B, N, H, S]
     int N, S, H;
     int num_kb;            // key blocks of 128
+    int num_qb;            // query blocks of 128
+    int num_np;            // n pairs, ceil(N / 2)
     float scale_log2;      // log2(e) / sqrt(D)
 };
 
 constexpr int kBM = 128;          // query rows per slice tile
 constexpr int kBN = 128;          // keys per block
-constexpr int kThreads = 384;
+constexpr int kThreads = 608;          // 3 helper warps + 16 softmax warps (104 registers each)
+constexpr int kFirstSoftmaxWarp = 3;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p <= 2^8 between rescales
@@ -70,23 +94,26 @@ struct Bf16Cfg {
     static_assert(D == 16 || D == 32 || D == 64, "head dim");
     static constexpr int ROW = D * 2;                 // bytes per Q/K/V row = swizzle span
     static constexpr int TILE = kBM * ROW;            // one Q, K or V tile
+    static constexpr bool SUM_MMA = D <= 32;          // row sum from a ones column of V
+    static constexpr int OW = D + (SUM_MMA ? 16 : 0); // O accumulator columns
     static constexpr int K_STAGES = (D <= 32) ? 4 : 3;
     static constexpr int V_STAGES = (D <= 32) ? 4 : 3;
-    static constexpr int B_STAGES = HAS_PAIR ? 2 : 0;
+    static constexpr int V_STRIDE = SUM_MMA ? 2 * TILE : TILE;  // V tile (+ ones tile)
     static constexpr int M_STAGES = 2;
     static constexpr int BIAS_BYTES = kBM * kBN * 2;  // two 128x64 boxes, 128 B swizzle
+    static constexpr int B_STAGES = HAS_PAIR ? 2 : 0;
     // shared-memory map (offsets from a 1024-aligned base)
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + 2 * TILE;
     static constexpr int OFF_V = OFF_K + K_STAGES * TILE;
-    static constexpr int OFF_BIAS = OFF_V + V_STAGES * TILE;
+    static constexpr int OFF_BIAS = OFF_V + V_STAGES * V_STRIDE;
     static constexpr int OFF_MASK = OFF_BIAS + B_STAGES * BIAS_BYTES;  // [2][M_STAGES][128] f32
     static constexpr int OFF_BAR = OFF_MASK + 2 * M_STAGES * kBN * 4;
     // barrier indices
     static constexpr int BAR_Q = 0;
     static constexpr int BAR_KF = 1;
     static constexpr int BAR_KE = BAR_KF + K_STAGES;
-    static constexpr int BAR_VF = BAR_KE + K_STAGES;
+    static constexpr int BAR_VF = BAR_KE + K_STAGES;   // V landed (bf16)
     static constexpr int BAR_VE = BAR_VF + V_STAGES;
     static constexpr int BAR_BF = BAR_VE + V_STAGES;
     static constexpr int BAR_BE = BAR_BF + 2;
@@ -107,13 +134,16 @@ struct Bf16Cfg {
     // tensor-memory columns
     static constexpr uint32_t TM_S0 = 0;    // + 128 * w
     static constexpr uint32_t TM_P0 = 256;  // + 64 * w
-    static constexpr uint32_t TM_O0 = 384;  // + D * w
+    static constexpr uint32_t TM_O0 = 384;  // + OW * w
     static constexpr uint32_t TMEM_COLS = 512;
-    // instruction descriptors: fp32 accumulate, bf16 A and B, M = 128
+    static_assert(TM_O0 + 2 * OW <= TMEM_COLS, "tensor memory");
+    // instruction descriptors, fp32 accumulate, M = 128:
+    // Q K^T: bf16 x bf16, both K-major, N = 128 keys
     static constexpr uint32_t IDESC_QK =
         (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(kBN) >> 3) << 17) | ((uint32_t(kBM) >> 4) << 24);
-    static constexpr uint32_t IDESC_PV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
-                                         ((uint32_t(D) >> 3) << 17) | ((uint32_t(kBM) >> 4) << 24);
+    // P V: fp16 x fp16, P from tensor memory, V MN-major, N = OW
+    static constexpr uint32_t IDESC_PV =
+        (1u << 4) | (0u << 7) | (0u << 10) | (1u << 16) | ((uint32_t(OW) >> 3) << 17) | ((uint32_t(kBM) >> 4) << 24);
 };
 
 // K-major operand tile: rows of ROW bytes, swizzled over ROW bytes, 8-row
@@ -129,17 +159,61 @@ __device__ __forceinline__ uint64_t desc_k_major(uint32_t saddr) {
     return d;
 }
 
-// MN-major operand tile (V as the B operand of P.V: N = D contiguous, K = keys
-// along rows): one swizzle atom spans all D columns; 8-key groups ROW*8 apart.
+// MN-major operand (V as the B operand of P.V: N = head dim contiguous, K =
+// keys along rows).  One swizzle atom spans ROW bytes of N; the next atom of N
+// (the ones tile) is `atom_stride` bytes further; 8-key groups are ROW*8 apart.
 template <int ROW>
-__device__ __forceinline__ uint64_t desc_mn_major(uint32_t saddr, uint32_t tile_bytes) {
+__device__ __forceinline__ uint64_t desc_mn_major(uint32_t saddr, uint32_t atom_stride) {
     uint64_t d = 0;
     d |= uint64_t((saddr >> 4) & 0x3FFFu);
-    d |= uint64_t((tile_bytes >> 4) & 0x3FFFu) << 16;        // next MN atom (none here)
-    d |= uint64_t(((8u * ROW) >> 4) & 0x3FFFu) << 32;        // stride between 8-key groups
+    d |= uint64_t((atom_stride >> 4) & 0x3FFFu) << 16;
+    d |= uint64_t(((8u * ROW) >> 4) & 0x3FFFu) << 32;
     d |= uint64_t(1) << 46;
     d |= uint64_t(umma_layout_code(ROW)) << 61;
     return d;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Converts 16 rows (keys) of a TMA-swizzled bf16 V tile to fp16 in place and
+// swaps rows 4g+1 and 4g+2 of every group of four (the key order in which the
+// softmax packs P).  Row r's 16-byte chunk c sits at chunk c ^ ((r * ROW /
+// 128) % (ROW / 16)) of the row.  A value beyond the fp16 range becomes
+// +-inf and surfaces as a non-finite row sum or output, which the epilogue
+// reports as EVO_ERR_RANGE.
+template <int ROW>
+__device__ __forceinline__ void convert_v_rows(uint32_t tile, int row0, int lane) {
+    constexpr int CHUNKS = ROW / 16;              // 16 B chunks per row
+    constexpr int ITEMS = 16 * CHUNKS;            // 16 rows x CHUNKS, spread over the warp
+    constexpr int PER_LANE = (ITEMS + 31) / 32;
+    auto at = [&](int r, int c) -> uint32_t {
+        const int sw = ((r * ROW) >> 7) & (CHUNKS - 1);
+        return tile + uint32_t(r * ROW) + uint32_t((c ^ sw) << 4);
+    };
+    uint4 v[PER_LANE];
+#pragma unroll
+    for (int k = 0; k < PER_LANE; ++k) {
+        const int item = lane + 32 * k;
+        if (item < ITEMS) v[k] = ptx::ld_shared_v4(at(row0 + item / CHUNKS, item % CHUNKS));
+    }
+    __syncwarp();  // every lane has read before any lane overwrites a swapped row
+#pragma unroll
+    for (int k = 0; k < PER_LANE; ++k) {
+        const int item = lane + 32 * k;
+        if (item < ITEMS) {
+            const int rr = item / CHUNKS;
+            const int dst = (rr & ~3) | ((rr & 1) << 1) | ((rr >> 1) & 1);  // swap rows 1 and 2 of each 4
+            uint32_t o[4];
+            const uint32_t wv[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[e] = ptx::pack_f16x2(ptx::bf16lo_to_f32(wv[e]), ptx::bf16hi_to_f32(wv[e]));
+            ptx::st_shared_v4(at(row0 + dst, item % CHUNKS), make_uint4(o[0], o[1], o[2], o[3]));
+        }
+    }
 }
 
 template <int D, bool HAS_PAIR>
@@ -154,11 +228,17 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * 2;
-    const int q0 = blockIdx.y * kBM;
-    const int bh = blockIdx.z;
-    const int b = bh / p.H;
-    const int h = bh - b * p.H;
+    // CTA index: query block fastest, then head, then n pair, then batch
+    int rest = blockIdx.x;
+    const int qb = rest % p.num_qb;
+    rest /= p.num_qb;
+    const int h = rest % p.H;
+    rest /= p.H;
+    const int np = rest % p.num_np;
+    const int b = rest / p.num_np;
+    const int n0 = np * 2;
+    const int q0 = qb * kBM;
+    const int bh = b * p.H + h;
     const int n_valid = (p.N - n0) < 2 ? (p.N - n0) : 2;
     const int nkb = p.num_kb;
 
@@ -179,16 +259,16 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(bar(C::BAR_BF + s), 1);
-            ptx::mbar_init(bar(C::BAR_BE + s), 4 * n_valid);
+            ptx::mbar_init(bar(C::BAR_BE + s), 8 * n_valid);
         }
         for (int s = 0; s < 2 * C::M_STAGES; ++s) {
             ptx::mbar_init(bar(C::BAR_MF + s), 32);
-            ptx::mbar_init(bar(C::BAR_ME + s), 4);
+            ptx::mbar_init(bar(C::BAR_ME + s), 8);
         }
         for (int w = 0; w < 2; ++w) {
             ptx::mbar_init(bar(C::BAR_SF + w), 1);
-            ptx::mbar_init(bar(C::BAR_SE + w), 4);
-            ptx::mbar_init(bar(C::BAR_PF + w), 4);
+            ptx::mbar_init(bar(C::BAR_SE + w), 8);
+            ptx::mbar_init(bar(C::BAR_PF + w), 8);
             ptx::mbar_init(bar(C::BAR_PE + w), 1);
         }
         ptx::mbar_init(bar(C::BAR_DRAIN), 1);
@@ -196,6 +276,26 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         csub_s[0] = 0.f;
         csub_s[1] = 0.f;
         ptx::fence_mbar_init();
+    }
+    if (C::SUM_MMA && warp == 2) {
+        // Constant tiles after each V stage: column 0 = 1.0 (fp16), rest 0,
+        // laid out with the same swizzle as V (16 B chunk c of row r sits at
+        // chunk c ^ ((r * ROW / 128) % (ROW / 16))).
+        for (int s = 0; s < C::V_STAGES; ++s) {
+            const uint32_t base = sb + C::OFF_V + uint32_t(s * C::V_STRIDE + C::TILE);
+            for (int c = lane; c < C::TILE / 16; c += 32)
+                ptx::st_shared_v4(base + uint32_t(c) * 16u, make_uint4(0u, 0u, 0u, 0u));
+        }
+        __syncwarp();
+        for (int s = 0; s < C::V_STAGES; ++s) {
+            const uint32_t base = sb + C::OFF_V + uint32_t(s * C::V_STRIDE + C::TILE);
+            for (int r = lane; r < kBM; r += 32) {
+                const uint32_t chunk = uint32_t((r * C::ROW) >> 7) & uint32_t(C::ROW / 16 - 1);
+                asm volatile("st.shared.u16 [%0], %1;" ::"r"(base + uint32_t(r * C::ROW) + chunk * 16u),
+                             "h"(uint16_t(0x3C00)) : "memory");
+            }
+        }
+        ptx::fence_proxy_async_smem();
     }
     if (warp == 0) {
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), C::TMEM_COLS);
@@ -243,7 +343,8 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const uint32_t ph = (v_issued / C::V_STAGES) & 1;
                     if (!wait_bounded(bar(C::BAR_VE + s), ph ^ 1, abort_flag)) { ok = false; break; }
                     ptx::mbar_arrive_expect_tx(bar(C::BAR_VF + s), C::TILE);
-                    ptx::tma_load_4d(sb + C::OFF_V + s * C::TILE, &tm_v, bar(C::BAR_VF + s), 0, h, j * kBN, bn0 + w);
+                    ptx::tma_load_4d(sb + C::OFF_V + s * C::V_STRIDE, &tm_v, bar(C::BAR_VF + s), 0, h, j * kBN,
+                                     bn0 + w);
                     ++v_issued;
                 }
             }
@@ -267,7 +368,7 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             int k_used = 0, v_used = 0;
             auto issue_qk = [&](int w) -> bool {
                 const int s = k_used % C::K_STAGES;
-                if (!wait_bounded(bar(C::BAR_KF + s), (k_used / C::K_STAGES) & 1, abort_flag)) return false;
+                if (!wait_fast(bar(C::BAR_KF + s), (k_used / C::K_STAGES) & 1, abort_flag)) return false;
                 ptx::tc_fence_after();
                 const uint64_t a = desc_k_major<C::ROW>(sb + C::OFF_Q + w * C::TILE);
                 const uint64_t bdesc = desc_k_major<C::ROW>(sb + C::OFF_K + s * C::TILE);
@@ -283,20 +384,18 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int w = 0; w < n_valid && ok; ++w) ok = issue_qk(w);
             for (int j = 0; j < nkb && ok; ++j) {
                 if (j + 1 < nkb) {
-                    for (int w = 0; w < n_valid && ok; ++w) {
-                        ok = wait_bounded(bar(C::BAR_SE + w), j & 1, abort_flag) && issue_qk(w);
-                    }
+                    for (int w = 0; w < n_valid && ok; ++w)
+                        ok = wait_fast(bar(C::BAR_SE + w), j & 1, abort_flag) && issue_qk(w);
                 }
                 for (int w = 0; w < n_valid && ok; ++w) {
                     const int s = v_used % C::V_STAGES;
-                    ok = wait_bounded(bar(C::BAR_VF + s), (v_used / C::V_STAGES) & 1, abort_flag) &&
-                         wait_bounded(bar(C::BAR_PF + w), j & 1, abort_flag);
+                    ok = wait_fast(bar(C::BAR_PF + w), j & 1, abort_flag);  // P written and V converted
                     if (!ok) break;
                     ptx::tc_fence_after();
-                    const uint64_t bdesc = desc_mn_major<C::ROW>(sb + C::OFF_V + s * C::TILE, C::TILE);
+                    const uint64_t bdesc = desc_mn_major<C::ROW>(sb + C::OFF_V + s * C::V_STRIDE, C::TILE);
 #pragma unroll
                     for (int kk = 0; kk < kBN / 16; ++kk)  // 16 keys per K step = 16 rows of V
-                        ptx::mma_ts(tmem + C::TM_O0 + uint32_t(D) * w, tmem + C::TM_P0 + 64u * w + 8u * kk,
+                        ptx::mma_ts(tmem + C::TM_O0 + uint32_t(C::OW) * w, tmem + C::TM_P0 + 64u * w + 8u * kk,
                                     bdesc + uint64_t((16 * C::ROW * kk) >> 4), C::IDESC_PV,
                                     (j > 0 || kk > 0) ? 1u : 0u);
                     ptx::mma_commit(bar(C::BAR_VE + s));
@@ -312,7 +411,7 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         __syncwarp();
     } else if (warp == 2) {
-        // ---------------------------------------------------------- mask warp
+        // ------------------------------------------------------------ mask warp
         float csub[2] = {0.f, 0.f};
         const uint16_t* mrow[2] = {nullptr, nullptr};
         for (int w = 0; w < n_valid; ++w) {
@@ -332,6 +431,7 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const int stage = j % C::M_STAGES;
                 const uint32_t ph = (j / C::M_STAGES) & 1;
                 if (!wait_warp(bar(C::BAR_ME + w * C::M_STAGES + stage), ph ^ 1, abort_flag)) { ok = false; break; }
+                // even keys first, then odd keys: a softmax thread reads its own parity
                 float* dst = reinterpret_cast<float*>(smem + C::OFF_MASK) + (w * C::M_STAGES + stage) * kBN;
 #pragma unroll
                 for (int t = lane; t < kBN; t += 32) {
@@ -341,38 +441,44 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         const float m = mrow[w] ? __uint_as_float(uint32_t(mrow[w][key]) << 16) : 0.f;
                         v = (m - csub[w]) * kLog2e;
                     }
-                    dst[t] = v;
+                    dst[(t & 1) * (kBN / 2) + (t >> 1)] = v;
                 }
                 ptx::mbar_arrive(bar(C::BAR_MF + w * C::M_STAGES + stage));
             }
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    } else {
         // ------------------------------------------------------------ softmax
-        const int w = (warp - 4) >> 2;
-        const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;  // query row in the tile == TMEM lane
+        const int sidx = warp - kFirstSoftmaxWarp;  // 0..15
+        const int w = sidx >> 3;                    // slice (n0 + w)
+        const int quarter = warp & 3;               // this warp may touch TMEM lanes 32*quarter .. +31
+        const int sub = (sidx >> 2) & 1;            // which 16 of those 32 lanes
+        const int lane0 = quarter * 32 + sub * 16;  // first row of the warp
+        const int par = (lane >> 1) & 1;            // key parity this thread holds
+        const int r = lane0 + (lane >> 2) + 8 * (lane & 1);  // query row in the tile == TMEM lane
         if (w < n_valid) {
-            const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+            const uint32_t lane_base = uint32_t(lane0) << 16;
             const uint32_t tS = tmem + lane_base + C::TM_S0 + 128u * w;
             const uint32_t tP = tmem + lane_base + C::TM_P0 + 64u * w;
-            const uint32_t tO = tmem + lane_base + C::TM_O0 + uint32_t(D) * w;
+            const uint32_t tO = tmem + lane_base + C::TM_O0 + uint32_t(C::OW) * w;
+            const float2 l2e2 = make_float2(kLog2e, kLog2e);
+            const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+            const float2 one2 = make_float2(1.f, 1.f);
+            // byte selector that moves this thread's bf16 half of a word into the high half of a float
+            const uint32_t psel = par ? 0x3244u : 0x1044u;
             float m_used = -INFINITY;
-            float l = 0.f;
+            float l = 0.f;  // this thread's share of the row sum when the tensor core does not keep it
             bool ok = true;
             for (int j = 0; j < nkb; ++j) {
-                uint32_t s[128];
+                // s[i] = S[r][2i + par], i = 0..63
+                uint32_t s[64];
                 ok = wait_warp(bar(C::BAR_SF + w), j & 1, abort_flag);
                 if (!ok) break;
                 ptx::tc_fence_after();
-                ptx::tmem_ld_x32(tS + 0, s);
-                ptx::tmem_ld_x32(tS + 32, s + 32);
-                ptx::tmem_ld_x32(tS + 64, s + 64);
-                ptx::tmem_ld_x32(tS + 96, s + 96);
+                ptx::tmem_ld_16x64b_x32(tS + 0, s);
+                ptx::tmem_ld_16x64b_x32(tS + 64, s + 32);
                 ptx::tmem_ld_wait_x32(s);
                 ptx::reg_fence_x32(s + 32);
-                ptx::reg_fence_x32(s + 64);
-                ptx::reg_fence_x32(s + 96);
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(bar(C::BAR_SE + w));
@@ -385,38 +491,43 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ok = wait_warp(bar(C::BAR_BF + bstage), (j >> 1) & 1, abort_flag);
                     if (!ok) break;
                 }
-                const uint32_t maddr = sb + C::OFF_MASK + uint32_t((w * C::M_STAGES + mstage) * kBN * 4);
+                const uint32_t maddr = sb + C::OFF_MASK + uint32_t((w * C::M_STAGES + mstage) * kBN * 4) +
+                                       uint32_t(par * (kBN / 2) * 4);
                 const uint32_t brow = sb + C::OFF_BIAS + uint32_t(bstage * C::BIAS_BYTES) + uint32_t(r * 128);
-                float rmax = -INFINITY;
+                float rmax0 = -INFINITY, rmax1 = -INFINITY;
 #pragma unroll
-                for (int cc = 0; cc < 16; ++cc) {  // 8 keys per step
-                    const float4 m0 = ptx::ld_shared_f4(maddr + cc * 32);
-                    const float4 m1 = ptx::ld_shared_f4(maddr + cc * 32 + 16);
-                    float bias[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+                for (int c = 0; c < 16; ++c) {  // bias chunk c: keys 8c .. 8c+7, this thread's 4 of them
+                    const float4 mv = ptx::ld_shared_f4(maddr + c * 16);
+                    float2 t0 = make_float2(mv.x, mv.y), t1 = make_float2(mv.z, mv.w);
                     if (HAS_PAIR) {
-                        // 128 B swizzle: 16 B chunk c of row r sits at chunk c ^ (r % 8)
-                        const int box = cc >> 3, c = cc & 7;
-                        const uint4 pw = ptx::ld_shared_v4(brow + uint32_t(box * (C::BIAS_BYTES / 2)) +
-                                                           uint32_t(((c ^ (r & 7)) << 4)));
-                        const uint32_t wv[4] = {pw.x, pw.y, pw.z, pw.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            bias[2 * e] = fmaf(ptx::bf16lo_to_f32(wv[e]), kLog2e, bias[2 * e]);
-                            bias[2 * e + 1] = fmaf(ptx::bf16hi_to_f32(wv[e]), kLog2e, bias[2 * e + 1]);
-                        }
+                        // 128 B swizzle: chunk (c % 8) of row r in box c / 8 sits at chunk (c % 8) ^ (r % 8)
+                        const uint4 pw = ptx::ld_shared_v4(brow + uint32_t((c >> 3) * (C::BIAS_BYTES / 2)) +
+                                                           uint32_t((((c & 7) ^ (r & 7)) << 4)));
+                        const float b0 = __uint_as_float(__byte_perm(pw.x, 0u, psel));
+                        const float b1 = __uint_as_float(__byte_perm(pw.y, 0u, psel));
+                        const float b2 = __uint_as_float(__byte_perm(pw.z, 0u, psel));
+                        const float b3 = __uint_as_float(__byte_perm(pw.w, 0u, psel));
+                        t0 = __ffma2_rn(make_float2(b0, b1), l2e2, t0);
+                        t1 = __ffma2_rn(make_float2(b2, b3), l2e2, t1);
                     }
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float u = fmaf(__uint_as_float(s[cc * 8 + e]), p.scale_log2, bias[e]);
-                        s[cc * 8 + e] = __float_as_uint(u);
-                        rmax = fmaxf(rmax, u);
-                    }
+                    const int k = 4 * c;
+                    const float2 u0 = __ffma2_rn(make_float2(__uint_as_float(s[k]), __uint_as_float(s[k + 1])), sc2, t0);
+                    const float2 u1 =
+                        __ffma2_rn(make_float2(__uint_as_float(s[k + 2]), __uint_as_float(s[k + 3])), sc2, t1);
+                    s[k] = __float_as_uint(u0.x);
+                    s[k + 1] = __float_as_uint(u0.y);
+                    s[k + 2] = __float_as_uint(u1.x);
+                    s[k + 3] = __float_as_uint(u1.y);
+                    rmax0 = max3f(rmax0, u0.x, u0.y);
+                    rmax1 = max3f(rmax1, u1.x, u1.y);
                 }
                 __syncwarp();
                 if (lane == 0) {
                     ptx::mbar_arrive(bar(C::BAR_ME + w * C::M_STAGES + mstage));
                     if (HAS_PAIR) ptx::mbar_arrive(bar(C::BAR_BE + bstage));
                 }
+                float rmax = fmaxf(rmax0, rmax1);
+                rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 2));  // the other parity of the row
 
                 const float m_new = fmaxf(m_used, rmax);
                 const bool rescale = m_new > m_used + kRescaleThreshold;
@@ -426,16 +537,7 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     m_used = m_new;
                 }
                 const float m_safe = (m_used == -INFINITY) ? 0.f : m_used;
-                float rsum = 0.f;
-                uint32_t pk[64];
-#pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const float p0 = ptx::ex2_approx(__uint_as_float(s[2 * c]) - m_safe);
-                    const float p1 = ptx::ex2_approx(__uint_as_float(s[2 * c + 1]) - m_safe);
-                    rsum += p0 + p1;
-                    pk[c] = ptx::pack_bf16x2(p0, p1);
-                }
-                l = l * alpha + rsum;
+                const float2 nm2 = make_float2(-m_safe, -m_safe);
 
                 if (j > 0) {
                     // P and O of the previous block are in use until its P.V is done.
@@ -444,18 +546,45 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     ptx::tc_fence_after();
                     if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-                        for (int dc = 0; dc < D; dc += 16) {
-                            uint32_t o[16];
-                            ptx::tmem_ld_x16(tO + dc, o);
-                            ptx::tmem_ld_wait_x16(o);
+                        for (int dc = 0; dc < C::OW; dc += 16) {  // 8 repeats of 2 columns
+                            uint32_t o[8];
+                            ptx::tmem_ld_16x64b_x8(tO + dc, o);
+                            ptx::tmem_ld_wait_x8(o);
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                            ptx::tmem_st_x16(tO + dc, o);
+                            for (int e = 0; e < 8; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                            ptx::tmem_st_16x64b_x8(tO + dc, o);
                         }
                     }
                 }
-                ptx::tmem_st_x32(tP, pk);
-                ptx::tmem_st_x32(tP + 32, pk + 32);
+                float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    // register i of the store lands in P column 2i + par: it packs this
+                    // thread's keys 2(2i') + par and 2(2i'+1) + par (MMA key order 0,2,1,3)
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int k = 32 * half + 2 * c;
+                        const float2 x =
+                            __ffma2_rn(make_float2(__uint_as_float(s[k]), __uint_as_float(s[k + 1])), one2, nm2);
+                        const float p0 = ptx::ex2_approx(x.x);
+                        const float p1 = ptx::ex2_approx(x.y);
+                        if (!C::SUM_MMA) acc = __ffma2_rn(make_float2(p0, p1), one2, acc);
+                        pk[c] = ptx::pack_f16x2(p0, p1);
+                    }
+                    ptx::tmem_st_16x64b_x16(tP + 32 * half, pk);
+                }
+                if (!C::SUM_MMA) l = l * alpha + (acc.x + acc.y);
+
+                // this warp's 16 rows of V_j for slice w: bf16 -> fp16 in place, key order 0,2,1,3
+                {
+                    const int vi = j * n_valid + w;  // index of the tile in the producer's V order
+                    const int vs = vi % C::V_STAGES;
+                    ok = wait_warp(bar(C::BAR_VF + vs), (vi / C::V_STAGES) & 1, abort_flag);
+                    if (!ok) break;
+                    convert_v_rows<C::ROW>(sb + C::OFF_V + uint32_t(vs * C::V_STRIDE), 16 * (sidx & 7), lane);
+                    ptx::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+                }
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
                 __syncwarp();
@@ -467,28 +596,57 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ptx::tc_fence_after();
                 const int n = n0 + w;
                 const int row = q0 + r;
+                if (C::SUM_MMA) {
+                    uint32_t o[8];
+                    ptx::tmem_ld_16x64b_x8(tO + D, o);  // column D (even) holds the row sum
+                    ptx::tmem_ld_wait_x8(o);
+                    l = __uint_as_float(o[0]);
+                    l = __shfl_sync(0xffffffffu, l, lane & ~2);  // from the even-column thread
+                } else {
+                    l += __shfl_xor_sync(0xffffffffu, l, 2);
+                }
                 const float inv_l = l > 0.f ? 1.f / l : 0.f;
-                uint16_t* orow = p.out + ((size_t(b) * p.N + n) * size_t(p.S) + size_t(row)) * size_t(p.H) * D +
-                                 size_t(h) * D;
+                // thread (row, par) holds d = 2i + par; swap halves with the partner so that
+                // par 0 stores d in [0, D/2) and par 1 stores d in [D/2, D)
+                constexpr int NV = D / 2;  // values per thread
+                uint32_t o[NV];
 #pragma unroll
                 for (int dc = 0; dc < D; dc += 16) {
-                    uint32_t o[16];
-                    ptx::tmem_ld_x16(tO + dc, o);
-                    ptx::tmem_ld_wait_x16(o);
-                    uint32_t packed[8];
+                    ptx::tmem_ld_16x64b_x8(tO + dc, o + dc / 2);
+                }
+                ptx::tmem_ld_wait_x8(o);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        packed[e] = ptx::pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
-                                                     __uint_as_float(o[2 * e + 1]) * inv_l);
-                    if (row < p.S) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + dc);
-                        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-                    }
+                for (int i = 8; i < NV; i += 8) ptx::reg_fence_x8(o + i);
+                bool finite = (l < INFINITY);  // an fp16 overflow of V shows up here or in O
+                // value i holds d = 2i + par.  par 0 stores d in [0, NV): its own even d and the
+                // partner's odd d of slots 0..NV/2-1; par 1 stores d in [NV, D) from slots NV/2..NV-1.
+                float mine[NV];
+#pragma unroll
+                for (int k = 0; k < NV / 2; ++k) {
+                    const float lo = __uint_as_float(o[k]) * inv_l;           // d = 2k + par
+                    const float hi = __uint_as_float(o[k + NV / 2]) * inv_l;  // d = 2k + NV + par
+                    finite = finite && fabsf(lo) < INFINITY && fabsf(hi) < INFINITY;
+                    const float recv = __shfl_xor_sync(0xffffffffu, par ? lo : hi, 2);
+                    mine[2 * k] = par ? recv : lo;
+                    mine[2 * k + 1] = par ? hi : recv;
                 }
                 if (row < p.S) {
-                    const float lse = l > 0.f ? (m_used + ptx::lg2_approx(l)) * kLn2 + csub_s[w] : -INFINITY;
-                    p.lse[((size_t(b) * p.N + n) * p.H + h) * size_t(p.S) + row] = lse;
+                    uint16_t* orow = p.out + ((size_t(b) * p.N + n) * size_t(p.S) + size_t(row)) * size_t(p.H) * D +
+                                     size_t(h) * D + size_t(NV * par);
+#pragma unroll
+                    for (int k = 0; k < NV; k += 8) {
+                        uint4 v;
+                        v.x = ptx::pack_bf16x2(mine[k + 0], mine[k + 1]);
+                        v.y = ptx::pack_bf16x2(mine[k + 2], mine[k + 3]);
+                        v.z = ptx::pack_bf16x2(mine[k + 4], mine[k + 5]);
+                        v.w = ptx::pack_bf16x2(mine[k + 6], mine[k + 7]);
+                        *reinterpret_cast<uint4*>(orow + k) = v;
+                    }
+                    if (!finite) record_status(EVO_ERR_RANGE);
+                    if (par == 0) {
+                        const float lse = l > 0.f ? (m_used + ptx::lg2_approx(l)) * kLn2 + csub_s[w] : -INFINITY;
+                        p.lse[((size_t(b) * p.N + n) * p.H + h) * size_t(p.S) + row] = lse;
+                    }
                 }
             }
         }

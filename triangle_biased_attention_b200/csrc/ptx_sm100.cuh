@@ -173,6 +173,8 @@ __device__ __forceinline__ void tmem_ld_wait_x16(uint32_t* r) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" : EVO_P8(0), EVO_P8(8) : : "memory");
 }
 
+__device__ __forceinline__ void reg_fence_x8(uint32_t* r) { asm volatile("" : EVO_P8(0) : : "memory"); }
+
 // Orders later uses of 32 more registers after a preceding wait (no instruction).
 __device__ __forceinline__ void reg_fence_x32(uint32_t* r) {
     asm volatile("" : EVO_P8(0), EVO_P8(8), EVO_P8(16), EVO_P8(24) : : "memory");
@@ -187,6 +189,49 @@ __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t* r) {
         : "memory");
 }
 
+// 16-lane shapes: a warp covers 16 TMEM lanes; in .16x64b thread t holds
+// lane (t >> 2) + 8 * (t & 1) of the group and, for repeat i, the 32-bit
+// column 2 * i + ((t >> 1) & 1).  Lanes t and t ^ 2 therefore share a lane.
+__device__ __forceinline__ void tmem_ld_16x64b_x32(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x64b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : EVO_R8(0), EVO_R8(8), EVO_R8(16), EVO_R8(24)
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_16x64b_x16(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x64b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : EVO_R8(0), EVO_R8(8)
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_16x64b_x8(uint32_t taddr, uint32_t* r) {
+    asm volatile("tcgen05.ld.sync.aligned.16x64b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : EVO_R8(0)
+                 : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait_x8(uint32_t* r) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : EVO_P8(0) : : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_16x64b_x16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x64b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        EVO_I8(0), EVO_I8(8)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_16x64b_x8(uint32_t taddr, const uint32_t* r) {
+    asm volatile("tcgen05.st.sync.aligned.16x64b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), EVO_I8(0)
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* r) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -194,6 +239,7 @@ __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* r) {
         EVO_I8(0), EVO_I8(8)
         : "memory");
 }
+
 
 __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -224,6 +270,11 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
 __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
     float4 v;
     asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -240,6 +291,13 @@ __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_fl
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two floats -> fp16 pair, round to nearest even; `lo` lands in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
 
