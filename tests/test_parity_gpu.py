@@ -83,6 +83,8 @@ BF16_SHAPES = [
     (1, 2, 300, 2, 32, False, "tail", 2, 0.0),     # S not a multiple of 8, all n masked
     (1, 4, 256, 2, 32, True, "tail", 0, 0.01),     # peaky pair bias (+8 spikes)
     (1, 2, 512, 2, 64, True, "bernoulli", 0, 0.01),
+    (1, 3, 640, 2, 32, True, "head", 1, 0.0),      # leading blocks fully masked, then not
+    (1, 2, 520, 1, 16, False, "head", 0, 0.0),     # same without pair bias, ragged S
 ]
 
 

@@ -47,7 +47,10 @@
 //    moved when the block maximum exceeds it by more than 8 (p <= 256, exact
 //    after the final division by the row sum); moving it rescales O in
 //    tensor memory.
-//  * Mask rebase: c[b,n] = max_j mask[b,n,j] is subtracted from the mask and
+//  * Mask rebase: the mask warp keeps c = the largest mask value seen so far
+//    for each slice (an online max over key blocks), hands the softmax
+//    (mask - c) * log2(e), and publishes c with every block; when c grows the
+//    softmax lowers its running max by the same amount, and the final c is
 //    added back to the LSE.  The guide builds masks as 1e9*(mask-1) (section
 //    5.2); for an n whose every key is masked that is a constant shift of the
 //    row, and the rebase keeps fp32 from rounding every logit to -1e9.
@@ -108,7 +111,8 @@ struct Bf16Cfg {
     static constexpr int OFF_V = OFF_K + K_STAGES * TILE;
     static constexpr int OFF_BIAS = OFF_V + V_STAGES * V_STRIDE;
     static constexpr int OFF_MASK = OFF_BIAS + B_STAGES * BIAS_BYTES;  // [2][M_STAGES][128] f32
-    static constexpr int OFF_BAR = OFF_MASK + 2 * M_STAGES * kBN * 4;
+    static constexpr int OFF_MC = OFF_MASK + 2 * M_STAGES * kBN * 4;  // [2][M_STAGES] f32 rebase c
+    static constexpr int OFF_BAR = OFF_MC + 64;
     // barrier indices
     static constexpr int BAR_Q = 0;
     static constexpr int BAR_KF = 1;
@@ -125,7 +129,7 @@ struct Bf16Cfg {
     static constexpr int BAR_PE = BAR_PF + 2;
     static constexpr int BAR_DRAIN = BAR_PE + 2;
     static constexpr int NUM_BARS = BAR_DRAIN + 1;
-    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag, c[2]
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag
     static constexpr int USED = OFF_MISC + 16;
     // Request at least 116 KB so that two CTAs never share an SM: each CTA
     // allocates all 512 tensor-memory columns.
@@ -185,36 +189,45 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 // 128) % (ROW / 16)) of the row.  A value beyond the fp16 range becomes
 // +-inf and surfaces as a non-finite row sum or output, which the epilogue
 // reports as EVO_ERR_RANGE.
+// The 16 B chunks of V a softmax warp converts: rows row0 .. row0+15 of the
+// tile, spread over the lanes.  Offsets are computed once per thread.
 template <int ROW>
-__device__ __forceinline__ void convert_v_rows(uint32_t tile, int row0, int lane) {
-    constexpr int CHUNKS = ROW / 16;              // 16 B chunks per row
-    constexpr int ITEMS = 16 * CHUNKS;            // 16 rows x CHUNKS, spread over the warp
-    constexpr int PER_LANE = (ITEMS + 31) / 32;
-    auto at = [&](int r, int c) -> uint32_t {
-        const int sw = ((r * ROW) >> 7) & (CHUNKS - 1);
-        return tile + uint32_t(r * ROW) + uint32_t((c ^ sw) << 4);
-    };
-    uint4 v[PER_LANE];
-#pragma unroll
-    for (int k = 0; k < PER_LANE; ++k) {
-        const int item = lane + 32 * k;
-        if (item < ITEMS) v[k] = ptx::ld_shared_v4(at(row0 + item / CHUNKS, item % CHUNKS));
+struct VConvPlan {
+    static constexpr int CHUNKS = ROW / 16;            // 16 B chunks per row
+    static constexpr int ITEMS = 16 * CHUNKS;          // 16 rows x CHUNKS
+    static constexpr int PER_LANE = (ITEMS + 31) / 32;
+    uint32_t src[PER_LANE], dst[PER_LANE];
+    __device__ __forceinline__ static uint32_t at(int r, int c) {
+        const int sw = ((r * ROW) >> 7) & (CHUNKS - 1);  // row r's chunk c sits at chunk c ^ sw
+        return uint32_t(r * ROW) + uint32_t((c ^ sw) << 4);
     }
-    __syncwarp();  // every lane has read before any lane overwrites a swapped row
+    __device__ __forceinline__ VConvPlan(int row0, int lane) {
 #pragma unroll
-    for (int k = 0; k < PER_LANE; ++k) {
-        const int item = lane + 32 * k;
-        if (item < ITEMS) {
-            const int rr = item / CHUNKS;
-            const int dst = (rr & ~3) | ((rr & 1) << 1) | ((rr >> 1) & 1);  // swap rows 1 and 2 of each 4
+        for (int k = 0; k < PER_LANE; ++k) {
+            const int item = (lane + 32 * k) % ITEMS;  // lanes past the end redo an item (same result)
+            const int rr = item / CHUNKS, c = item % CHUNKS;
+            const int swapped = (rr & ~3) | ((rr & 1) << 1) | ((rr >> 1) & 1);  // rows 1 and 2 of each 4
+            src[k] = at(row0 + rr, c);
+            dst[k] = at(row0 + swapped, c);
+        }
+    }
+    // Converts bf16 -> fp16 in place with the row swap.  Every lane reads all its
+    // chunks before any lane writes.
+    __device__ __forceinline__ void run(uint32_t tile) const {
+        uint4 v[PER_LANE];
+#pragma unroll
+        for (int k = 0; k < PER_LANE; ++k) v[k] = ptx::ld_shared_v4(tile + src[k]);
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < PER_LANE; ++k) {
             uint32_t o[4];
             const uint32_t wv[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[e] = ptx::pack_f16x2(ptx::bf16lo_to_f32(wv[e]), ptx::bf16hi_to_f32(wv[e]));
-            ptx::st_shared_v4(at(row0 + dst, item % CHUNKS), make_uint4(o[0], o[1], o[2], o[3]));
+            ptx::st_shared_v4(tile + dst[k], make_uint4(o[0], o[1], o[2], o[3]));
         }
     }
-}
+};
 
 template <int D, bool HAS_PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -245,7 +258,7 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8u * uint32_t(i); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-    float* csub_s = reinterpret_cast<float*>(smem + C::OFF_MISC + 8);
+    float* mc_s = reinterpret_cast<float*>(smem + C::OFF_MC);  // [w * M_STAGES + stage]
 
     if (threadIdx.x == 0) {
         ptx::mbar_init(bar(C::BAR_Q), 1);
@@ -273,8 +286,6 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         ptx::mbar_init(bar(C::BAR_DRAIN), 1);
         *abort_flag = 0;
-        csub_s[0] = 0.f;
-        csub_s[1] = 0.f;
         ptx::fence_mbar_init();
     }
     if (C::SUM_MMA && warp == 2) {
@@ -412,37 +423,58 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         __syncwarp();
     } else if (warp == 2) {
         // ------------------------------------------------------------ mask warp
-        float csub[2] = {0.f, 0.f};
+        // Lane l handles keys l, l+32, l+64, l+96 of each block, for both slices;
+        // the next block's raw values are fetched while this block is processed.
+        // With a pair bias it also waits for the block's bias tile before
+        // releasing the stage, so one barrier tells a softmax warp both are ready.
         const uint16_t* mrow[2] = {nullptr, nullptr};
-        for (int w = 0; w < n_valid; ++w) {
-            if (p.mask != nullptr) {
-                mrow[w] = p.mask + (size_t(b) * p.N + n0 + w) * size_t(p.S);
-                float mx = -INFINITY;
-                for (int j = lane; j < p.S; j += 32) mx = fmaxf(mx, __uint_as_float(uint32_t(mrow[w][j]) << 16));
+        for (int w = 0; w < n_valid; ++w)
+            if (p.mask != nullptr) mrow[w] = p.mask + (size_t(b) * p.N + n0 + w) * size_t(p.S);
+        float c_run[2] = {-INFINITY, -INFINITY};
+        uint32_t raw[2][4];
+        auto fetch = [&](int j) {
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                csub[w] = (mx == -INFINITY) ? 0.f : mx;  // all -inf: leave -inf logits, LSE = -inf
-            }
-            if (lane == 0) csub_s[w] = csub[w];
-        }
+            for (int w = 0; w < 2; ++w)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int key = j * kBN + lane + 32 * k;
+                    raw[w][k] = (mrow[w] != nullptr && key < p.S) ? uint32_t(mrow[w][key]) : 0u;
+                }
+        };
+        fetch(0);
         bool ok = true;
         for (int j = 0; j < nkb && ok; ++j) {
+            uint32_t cur[2][4];
+#pragma unroll
+            for (int w = 0; w < 2; ++w)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) cur[w][k] = raw[w][k];
+            if (j + 1 < nkb) fetch(j + 1);
+            const int stage = j % C::M_STAGES;
+            const uint32_t ph = (j / C::M_STAGES) & 1;
+            if (HAS_PAIR && !wait_warp(bar(C::BAR_BF + (j & 1)), (j >> 1) & 1, abort_flag)) { ok = false; break; }
             for (int w = 0; w < n_valid && ok; ++w) {
-                const int stage = j % C::M_STAGES;
-                const uint32_t ph = (j / C::M_STAGES) & 1;
+                float v[4];
+                float bmax = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int key = j * kBN + lane + 32 * k;
+                    v[k] = key < p.S ? __uint_as_float(cur[w][k] << 16) : -INFINITY;  // absent mask: 0
+                    bmax = fmaxf(bmax, v[k]);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
+                c_run[w] = fmaxf(c_run[w], bmax);
+                const float csub = (c_run[w] == -INFINITY) ? 0.f : c_run[w];  // all -inf so far: keep -inf logits
                 if (!wait_warp(bar(C::BAR_ME + w * C::M_STAGES + stage), ph ^ 1, abort_flag)) { ok = false; break; }
                 // even keys first, then odd keys: a softmax thread reads its own parity
                 float* dst = reinterpret_cast<float*>(smem + C::OFF_MASK) + (w * C::M_STAGES + stage) * kBN;
 #pragma unroll
-                for (int t = lane; t < kBN; t += 32) {
-                    const int key = j * kBN + t;
-                    float v = -INFINITY;
-                    if (key < p.S) {
-                        const float m = mrow[w] ? __uint_as_float(uint32_t(mrow[w][key]) << 16) : 0.f;
-                        v = (m - csub[w]) * kLog2e;
-                    }
-                    dst[(t & 1) * (kBN / 2) + (t >> 1)] = v;
+                for (int k = 0; k < 4; ++k) {
+                    const int t = lane + 32 * k;
+                    dst[(t & 1) * (kBN / 2) + (t >> 1)] = (v[k] - csub) * kLog2e;
                 }
+                if (lane == 0) mc_s[w * C::M_STAGES + stage] = csub;
                 ptx::mbar_arrive(bar(C::BAR_MF + w * C::M_STAGES + stage));
             }
         }
@@ -466,8 +498,10 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const float2 one2 = make_float2(1.f, 1.f);
             // byte selector that moves this thread's bf16 half of a word into the high half of a float
             const uint32_t psel = par ? 0x3244u : 0x1044u;
+            const VConvPlan<C::ROW> vplan(16 * (sidx & 7), lane);
             float m_used = -INFINITY;
-            float l = 0.f;  // this thread's share of the row sum when the tensor core does not keep it
+            float c_cur = 0.f;  // mask rebase the current m_used and P are relative to
+            float l = 0.f;      // this thread's share of the row sum when the tensor core does not keep it
             bool ok = true;
             for (int j = 0; j < nkb; ++j) {
                 // s[i] = S[r][2i + par], i = 0..63
@@ -475,25 +509,28 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ok = wait_warp(bar(C::BAR_SF + w), j & 1, abort_flag);
                 if (!ok) break;
                 ptx::tc_fence_after();
-                ptx::tmem_ld_16x64b_x32(tS + 0, s);
-                ptx::tmem_ld_16x64b_x32(tS + 64, s + 32);
-                ptx::tmem_ld_wait_x32(s);
-                ptx::reg_fence_x32(s + 32);
+                ptx::tmem_ld_16x64b_x64_wait(tS, s);
                 ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(C::BAR_SE + w));
+                ptx::mbar_arrive_elect(bar(C::BAR_SE + w));
 
+                // mask vector (and, with a pair bias, the bias tile: the mask warp waited for it)
                 const int mstage = j % C::M_STAGES;
                 ok = wait_warp(bar(C::BAR_MF + w * C::M_STAGES + mstage), (j / C::M_STAGES) & 1, abort_flag);
                 if (!ok) break;
                 const int bstage = j & 1;
-                if (HAS_PAIR) {
-                    ok = wait_warp(bar(C::BAR_BF + bstage), (j >> 1) & 1, abort_flag);
-                    if (!ok) break;
+                {
+                    // the mask rebase grew: earlier logits are relative to a smaller c
+                    const float cs = mc_s[w * C::M_STAGES + mstage];
+                    if (cs != c_cur) {
+                        m_used -= (cs - c_cur) * kLog2e;
+                        c_cur = cs;
+                    }
                 }
                 const uint32_t maddr = sb + C::OFF_MASK + uint32_t((w * C::M_STAGES + mstage) * kBN * 4) +
                                        uint32_t(par * (kBN / 2) * 4);
-                const uint32_t brow = sb + C::OFF_BIAS + uint32_t(bstage * C::BIAS_BYTES) + uint32_t(r * 128);
+                // row r starts 128 B-aligned, so chunk k of it sits at (row start | (r % 8) << 4) ^ (k << 4)
+                const uint32_t brow = (sb + C::OFF_BIAS + uint32_t(bstage * C::BIAS_BYTES) + uint32_t(r * 128)) |
+                                      uint32_t((r & 7) << 4);
                 float rmax0 = -INFINITY, rmax1 = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {  // bias chunk c: keys 8c .. 8c+7, this thread's 4 of them
@@ -501,8 +538,8 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     float2 t0 = make_float2(mv.x, mv.y), t1 = make_float2(mv.z, mv.w);
                     if (HAS_PAIR) {
                         // 128 B swizzle: chunk (c % 8) of row r in box c / 8 sits at chunk (c % 8) ^ (r % 8)
-                        const uint4 pw = ptx::ld_shared_v4(brow + uint32_t((c >> 3) * (C::BIAS_BYTES / 2)) +
-                                                           uint32_t((((c & 7) ^ (r & 7)) << 4)));
+                        const uint4 pw =
+                            ptx::ld_shared_v4((brow ^ uint32_t((c & 7) << 4)) + uint32_t((c >> 3) * (C::BIAS_BYTES / 2)));
                         const float b0 = __uint_as_float(__byte_perm(pw.x, 0u, psel));
                         const float b1 = __uint_as_float(__byte_perm(pw.y, 0u, psel));
                         const float b2 = __uint_as_float(__byte_perm(pw.z, 0u, psel));
@@ -521,11 +558,8 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     rmax0 = max3f(rmax0, u0.x, u0.y);
                     rmax1 = max3f(rmax1, u1.x, u1.y);
                 }
-                __syncwarp();
-                if (lane == 0) {
-                    ptx::mbar_arrive(bar(C::BAR_ME + w * C::M_STAGES + mstage));
-                    if (HAS_PAIR) ptx::mbar_arrive(bar(C::BAR_BE + bstage));
-                }
+                ptx::mbar_arrive_elect(bar(C::BAR_ME + w * C::M_STAGES + mstage));
+                if (HAS_PAIR) ptx::mbar_arrive_elect(bar(C::BAR_BE + bstage));
                 float rmax = fmaxf(rmax0, rmax1);
                 rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 2));  // the other parity of the row
 
@@ -539,8 +573,24 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const float m_safe = (m_used == -INFINITY) ? 0.f : m_used;
                 const float2 nm2 = make_float2(-m_safe, -m_safe);
 
+                float2 acc = make_float2(0.f, 0.f);
+                // register i of a store lands in P column 2i + par: it packs this thread's keys
+                // 2(2i') + par and 2(2i'+1) + par (MMA key order 0, 2, 1, 3)
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float2 x =
+                        __ffma2_rn(make_float2(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), one2, nm2);
+                    const float p0 = ptx::ex2_approx(x.x);
+                    const float p1 = ptx::ex2_approx(x.y);
+                    if (!C::SUM_MMA) acc = __ffma2_rn(make_float2(p0, p1), one2, acc);
+                    pk[c] = ptx::pack_f16x2(p0, p1);
+                }
+                if (!C::SUM_MMA) l = l * alpha + (acc.x + acc.y);
+
                 if (j > 0) {
-                    // P and O of the previous block are in use until its P.V is done.
+                    // P and O of the previous block are in use until its P.V is done; the
+                    // exp pass above overlaps that MMA.
                     ok = wait_warp(bar(C::BAR_PE + w), (j - 1) & 1, abort_flag);
                     if (!ok) break;
                     ptx::tc_fence_after();
@@ -556,25 +606,8 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         }
                     }
                 }
-                float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    // register i of the store lands in P column 2i + par: it packs this
-                    // thread's keys 2(2i') + par and 2(2i'+1) + par (MMA key order 0,2,1,3)
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const int k = 32 * half + 2 * c;
-                        const float2 x =
-                            __ffma2_rn(make_float2(__uint_as_float(s[k]), __uint_as_float(s[k + 1])), one2, nm2);
-                        const float p0 = ptx::ex2_approx(x.x);
-                        const float p1 = ptx::ex2_approx(x.y);
-                        if (!C::SUM_MMA) acc = __ffma2_rn(make_float2(p0, p1), one2, acc);
-                        pk[c] = ptx::pack_f16x2(p0, p1);
-                    }
-                    ptx::tmem_st_16x64b_x16(tP + 32 * half, pk);
-                }
-                if (!C::SUM_MMA) l = l * alpha + (acc.x + acc.y);
+                ptx::tmem_st_16x64b_x16(tP, pk);
+                ptx::tmem_st_16x64b_x16(tP + 32, pk + 16);
 
                 // this warp's 16 rows of V_j for slice w: bf16 -> fp16 in place, key order 0,2,1,3
                 {
@@ -582,13 +615,12 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const int vs = vi % C::V_STAGES;
                     ok = wait_warp(bar(C::BAR_VF + vs), (vi / C::V_STAGES) & 1, abort_flag);
                     if (!ok) break;
-                    convert_v_rows<C::ROW>(sb + C::OFF_V + uint32_t(vs * C::V_STRIDE), 16 * (sidx & 7), lane);
+                    vplan.run(sb + C::OFF_V + uint32_t(vs * C::V_STRIDE));
                     ptx::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
                 }
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(C::BAR_PF + w));
+                ptx::mbar_arrive_elect(bar(C::BAR_PF + w));
             }
             // ---------------------------------------------------------- epilogue
             if (ok) ok = wait_warp(bar(C::BAR_PE + w), (nkb - 1) & 1, abort_flag);
@@ -644,7 +676,7 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                     if (!finite) record_status(EVO_ERR_RANGE);
                     if (par == 0) {
-                        const float lse = l > 0.f ? (m_used + ptx::lg2_approx(l)) * kLn2 + csub_s[w] : -INFINITY;
+                        const float lse = l > 0.f ? (m_used + ptx::lg2_approx(l)) * kLn2 + c_cur : -INFINITY;
                         p.lse[((size_t(b) * p.N + n) * p.H + h) * size_t(p.S) + row] = lse;
                     }
                 }

@@ -175,6 +175,32 @@ __device__ __forceinline__ void tmem_ld_wait_x16(uint32_t* r) {
 
 __device__ __forceinline__ void reg_fence_x8(uint32_t* r) { asm volatile("" : EVO_P8(0) : : "memory"); }
 
+// Two 16x64b loads of 32 columns each (TMEM columns c0 .. c0+63 of the warp's
+// 16 lanes) and the wait for them, in one statement: the registers are valid
+// when it returns.
+__device__ __forceinline__ void tmem_ld_16x64b_x64_wait(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x64b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.16x64b.x32.b32 "
+        "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : EVO_R8(0), EVO_R8(8), EVO_R8(16), EVO_R8(24), EVO_R8(32), EVO_R8(40), EVO_R8(48), EVO_R8(56)
+        : "r"(taddr), "r"(taddr + 64u)
+        : "memory");
+}
+
+// One lane of the (converged) warp arrives on the mbarrier; no branch.
+__device__ __forceinline__ void mbar_arrive_elect(uint32_t bar) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(bar)
+        : "memory");
+}
+
 // Orders later uses of 32 more registers after a preceding wait (no instruction).
 __device__ __forceinline__ void reg_fence_x32(uint32_t* r) {
     asm volatile("" : EVO_P8(0), EVO_P8(8), EVO_P8(16), EVO_P8(24) : : "memory");

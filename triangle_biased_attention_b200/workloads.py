@@ -170,8 +170,10 @@ def random_case(B: int, N: int, S: int, H: int, D: int, dtype: torch.dtype, seed
     """A free-form seeded case for parity tests at arbitrary shapes.
 
     mask: "none" (no mask tensor), "zero" (all keys kept), "tail" (random tail of
-    up to S//4 keys masked per n), "bernoulli" (~5% of (n, j) masked),
-    "neg_inf" (random ~10% of keys set to -inf instead of -1e9).
+    up to S//4 keys masked per n), "head" (a random head of S//4 .. S//2 keys
+    masked per n, so leading key blocks can be fully masked), "bernoulli" (~5%
+    of (n, j) masked), "neg_inf" (random ~10% of keys set to -inf instead of
+    -1e9).
     fully_masked: how many n slices get every key masked with -1e9.
     """
     rng = _rng(seed)
@@ -195,6 +197,11 @@ def random_case(B: int, N: int, S: int, H: int, D: int, dtype: torch.dtype, seed
                     t = int(tails[b, n])
                     if t:
                         keep[b, n, S - t:] = False
+        elif mask == "head":
+            heads = rng.integers(S // 4, S // 2 + 1, size=(B, N))
+            for b in range(B):
+                for n in range(N):
+                    keep[b, n, : int(heads[b, n])] = False
         elif mask == "bernoulli":
             keep = rng.random((B, N, S)) >= 0.05
         elif mask == "neg_inf":
