@@ -123,6 +123,19 @@ EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
  */
 EVO_API int evo_attn_sync_status(evo_stream_t stream);
 
+/*
+ * evo_attn_selftest_timeout — exercises the device-side failure path without
+ * faulting anything: launches one warp on `stream` that waits on an internal
+ * barrier that nothing ever completes, with a limit of `limit_ns`
+ * nanoseconds (1 .. 1e9).  The wait gives up, records EVO_ERR_TIMEOUT in the
+ * status word and the kernel ends normally; *result (a device int) is set to
+ * 0.  A following evo_attn_sync_status(stream) returns EVO_ERR_TIMEOUT and
+ * clears the word.  The guide has no counterpart; this is a diagnostic of this
+ * library's bounded waits.  Returns EVO_OK once launched, EVO_ERR_INVALID_ARG
+ * for a limit outside the range or a NULL / non-device result pointer.
+ */
+EVO_API int evo_attn_selftest_timeout(int64_t limit_ns, int* result, evo_stream_t stream);
+
 /* evo_attn_strerror — a static, human-readable string for a status code. */
 EVO_API const char* evo_attn_strerror(int status);
 

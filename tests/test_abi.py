@@ -118,3 +118,9 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(evo, "_LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError, match="no fallback"):
         evo.load_library()
+
+
+def test_selftest_timeout_rejects_bad_arguments(lib):
+    assert evo.evo_attn_selftest_timeout(0, 0x1000, None) == evo.EVO_ERR_INVALID_ARG
+    assert evo.evo_attn_selftest_timeout(2 * 10**9, 0x1000, None) == evo.EVO_ERR_INVALID_ARG
+    assert evo.evo_attn_selftest_timeout(10**6, None, None) == evo.EVO_ERR_INVALID_ARG

@@ -23,6 +23,7 @@ import torch
 
 __all__ = [
     "evo_attn", "evo_attn_fwd", "evo_attn_sync_status", "evo_attn_strerror", "evo_attn_version",
+    "evo_attn_selftest_timeout",
     "EvoAttnError", "library_path", "load_library",
     "EVO_DTYPE_BF16", "EVO_DTYPE_FP32",
     "EVO_OK", "EVO_ERR_INVALID_ARG", "EVO_ERR_UNSUPPORTED_DTYPE", "EVO_ERR_UNSUPPORTED_SHAPE",
@@ -77,6 +78,8 @@ def load_library():
     lib.evo_attn_strerror.restype = ctypes.c_char_p
     lib.evo_attn_version.argtypes = []
     lib.evo_attn_version.restype = i32
+    lib.evo_attn_selftest_timeout.argtypes = [i64, vp, vp]
+    lib.evo_attn_selftest_timeout.restype = i32
     _lib = lib
     return lib
 
@@ -97,6 +100,11 @@ def evo_attn_strerror(status: int) -> str:
 
 def evo_attn_version() -> int:
     return int(load_library().evo_attn_version())
+
+
+def evo_attn_selftest_timeout(limit_ns: int, result_ptr: int, stream: Optional[int] = None) -> int:
+    """Launch the bounded-wait self-test (see include/evo_attn.h); returns the status code."""
+    return int(load_library().evo_attn_selftest_timeout(limit_ns, result_ptr, stream))
 
 
 def _ptr(t: Optional[torch.Tensor]):

@@ -16,7 +16,20 @@ __device__ int g_status;
 // A wait on an internal barrier longer than this is treated as a hang.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 
+
 __device__ __forceinline__ void record_status(int code) { atomicCAS(&g_status, 0, code); }
+
+// Bounded wait with an explicit limit (the self-test uses a short one).
+__device__ __noinline__ bool wait_bounded_for(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (true) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (ptx::globaltimer_ns() - t0 > limit_ns) {
+            record_status(EVO_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
 
 // Waits for the given phase parity of an mbarrier.  Returns false, after
 // raising the CTA's abort flag and recording EVO_ERR_TIMEOUT, if the phase

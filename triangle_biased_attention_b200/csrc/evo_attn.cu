@@ -169,7 +169,35 @@ int launch_f32(int dev, const void* Q, const void* K, const void* V, const void*
     return cudaLaunchKernelEx(&cfg, evo::evo_fwd_f32_kernel, p) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
 
+// One warp initialises an mbarrier that expects one arrival, never arrives,
+// and waits on it with a short limit: the wait must give up, record
+// EVO_ERR_TIMEOUT and let the kernel finish.
+__global__ void selftest_timeout_kernel(uint64_t limit_ns, int* result) {
+    __shared__ __align__(8) uint64_t mbar;
+    const uint32_t bar = evo::ptx::smem_u32(&mbar);
+    if (threadIdx.x == 0) {
+        evo::ptx::mbar_init(bar, 1);
+        evo::ptx::fence_mbar_init();
+    }
+    __syncwarp();
+    const bool ok = evo::wait_bounded_for(bar, 0, limit_ns);
+    if (threadIdx.x == 0) *result = ok ? 1 : 0;
+}
+
 }  // namespace
+
+extern "C" EVO_API int evo_attn_selftest_timeout(int64_t limit_ns, int* result, evo_stream_t stream) {
+    if (limit_ns <= 0 || limit_ns > 1000000000ll || result == nullptr) return EVO_ERR_INVALID_ARG;
+    const int dev = select_device_of(result);
+    if (dev < 0) return dev;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, 1);
+    cfg.blockDim = dim3(32, 1, 1);
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    return cudaLaunchKernelEx(&cfg, selftest_timeout_kernel, uint64_t(limit_ns), result) == cudaSuccess
+               ? EVO_OK
+               : EVO_ERR_CUDA;
+}
 
 extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V, const void* mask_bias,
                             const void* pair_bias, void* O, float* LSE, int64_t B, int64_t N, int64_t S, int64_t H,

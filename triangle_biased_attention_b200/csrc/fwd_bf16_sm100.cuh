@@ -25,10 +25,14 @@
 //    softmax warp also converts 16 rows of its slice's V tile to fp16 before
 //    it reports P ready, so the P.V MMA that waits for P also finds V
 //    converted.
-//  * Tensor memory (512 columns): per slice, S = Q K^T (128 fp32 columns),
-//    P = softmax numerators as fp16 (64 columns) and the O accumulator.  S and
-//    P are separate so the next block's Q K^T can start as soon as the softmax
-//    has pulled S into registers.
+//  * Tensor memory (512 columns): one S = Q K^T buffer (128 fp32 columns)
+//    that the two slices take turns in, two P buffers per slice (softmax
+//    numerators as fp16, 64 columns each) and one O accumulator per slice.
+//    A slice's next Q K^T is issued as soon as the other slice has pulled its
+//    S into registers, which staggers the two slices by about half a block;
+//    with two P buffers a softmax warp writes block j+1's P while block j's
+//    P.V is still running, so no warp waits for the tensor core in the steady
+//    state (only a rare O rescale waits for the previous P.V).
 //  * P is packed from a thread's own (interleaved) columns, so within every
 //    group of four keys the MMA sees key order 0, 2, 1, 3; the V conversion
 //    swaps rows 1 and 2 of every group of four to match (a permutation of
@@ -123,11 +127,14 @@ struct Bf16Cfg {
     static constexpr int BAR_BE = BAR_BF + 2;
     static constexpr int BAR_MF = BAR_BE + 2;           // [2][M_STAGES]
     static constexpr int BAR_ME = BAR_MF + 2 * M_STAGES;
-    static constexpr int BAR_SF = BAR_ME + 2 * M_STAGES;  // [2]
-    static constexpr int BAR_SE = BAR_SF + 2;
-    static constexpr int BAR_PF = BAR_SE + 2;
-    static constexpr int BAR_PE = BAR_PF + 2;
-    static constexpr int BAR_DRAIN = BAR_PE + 2;
+    static constexpr int BAR_SF = BAR_ME + 2 * M_STAGES;  // [2] S of slice w ready
+    static constexpr int BAR_SE = BAR_SF + 2;             // [2] slice w has read S
+    // P ready / P.V done, one barrier per P buffer: a slice can be one block
+    // ahead of the MMA issuer, and block j and j + 1 use different barriers,
+    // so a wait on block j's phase never sees block j + 2's.
+    static constexpr int BAR_PF = BAR_SE + 2;             // [2 slices][2 buffers] P written, V converted
+    static constexpr int BAR_PE = BAR_PF + 4;             // [2 slices][2 buffers] P.V done
+    static constexpr int BAR_DRAIN = BAR_PE + 4;
     static constexpr int NUM_BARS = BAR_DRAIN + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem slot, abort flag
     static constexpr int USED = OFF_MISC + 16;
@@ -136,8 +143,8 @@ struct Bf16Cfg {
     static constexpr int SMEM_BYTES = (USED + 1024 > 116 * 1024) ? USED + 1024 : 116 * 1024;
     static_assert(USED + 1024 <= 227 * 1024, "shared memory");
     // tensor-memory columns
-    static constexpr uint32_t TM_S0 = 0;    // + 128 * w
-    static constexpr uint32_t TM_P0 = 256;  // + 64 * w
+    static constexpr uint32_t TM_S = 0;     // shared by both slices
+    static constexpr uint32_t TM_P0 = 128;  // + 64 * (2 * w + buffer)
     static constexpr uint32_t TM_O0 = 384;  // + OW * w
     static constexpr uint32_t TMEM_COLS = 512;
     static_assert(TM_O0 + 2 * OW <= TMEM_COLS, "tensor memory");
@@ -281,8 +288,10 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int w = 0; w < 2; ++w) {
             ptx::mbar_init(bar(C::BAR_SF + w), 1);
             ptx::mbar_init(bar(C::BAR_SE + w), 8);
-            ptx::mbar_init(bar(C::BAR_PF + w), 8);
-            ptx::mbar_init(bar(C::BAR_PE + w), 1);
+            ptx::mbar_init(bar(C::BAR_PF + 2 * w), 8);
+            ptx::mbar_init(bar(C::BAR_PF + 2 * w + 1), 8);
+            ptx::mbar_init(bar(C::BAR_PE + 2 * w), 1);
+            ptx::mbar_init(bar(C::BAR_PE + 2 * w + 1), 1);
         }
         ptx::mbar_init(bar(C::BAR_DRAIN), 1);
         *abort_flag = 0;
@@ -385,35 +394,39 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint64_t bdesc = desc_k_major<C::ROW>(sb + C::OFF_K + s * C::TILE);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)  // 16 bf16 = 32 B per K step
-                    ptx::mma_ss(tmem + C::TM_S0 + 128u * w, a + uint64_t(2 * kk), bdesc + uint64_t(2 * kk),
+                    ptx::mma_ss(tmem + C::TM_S, a + uint64_t(2 * kk), bdesc + uint64_t(2 * kk),
                                 C::IDESC_QK, kk > 0 ? 1u : 0u);
                 ptx::mma_commit(bar(C::BAR_KE + s));
                 ptx::mma_commit(bar(C::BAR_SF + w));
                 ++k_used;
                 return true;
             };
-            for (int w = 0; w < n_valid && ok; ++w) ok = issue_qk(w);
-            for (int j = 0; j < nkb && ok; ++j) {
-                if (j + 1 < nkb) {
-                    for (int w = 0; w < n_valid && ok; ++w)
-                        ok = wait_fast(bar(C::BAR_SE + w), j & 1, abort_flag) && issue_qk(w);
-                }
-                for (int w = 0; w < n_valid && ok; ++w) {
-                    const int s = v_used % C::V_STAGES;
-                    ok = wait_fast(bar(C::BAR_PF + w), j & 1, abort_flag);  // P written and V converted
-                    if (!ok) break;
-                    ptx::tc_fence_after();
-                    const uint64_t bdesc = desc_mn_major<C::ROW>(sb + C::OFF_V + s * C::V_STRIDE, C::TILE);
+            auto issue_pv = [&](int w, int j) -> bool {
+                const int s = v_used % C::V_STAGES;
+                // P of block j written and V converted (buffer j & 1, its (j >> 1)-th use)
+                if (!wait_fast(bar(C::BAR_PF + 2 * w + (j & 1)), (j >> 1) & 1, abort_flag)) return false;
+                ptx::tc_fence_after();
+                const uint64_t bdesc = desc_mn_major<C::ROW>(sb + C::OFF_V + s * C::V_STRIDE, C::TILE);
+                const uint32_t a_tmem = tmem + C::TM_P0 + 64u * uint32_t(2 * w + (j & 1));
 #pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)  // 16 keys per K step = 16 rows of V
-                        ptx::mma_ts(tmem + C::TM_O0 + uint32_t(C::OW) * w, tmem + C::TM_P0 + 64u * w + 8u * kk,
-                                    bdesc + uint64_t((16 * C::ROW * kk) >> 4), C::IDESC_PV,
-                                    (j > 0 || kk > 0) ? 1u : 0u);
-                    ptx::mma_commit(bar(C::BAR_VE + s));
-                    ptx::mma_commit(bar(C::BAR_PE + w));
-                    ++v_used;
-                }
+                for (int kk = 0; kk < kBN / 16; ++kk)  // 16 keys per K step = 16 rows of V
+                    ptx::mma_ts(tmem + C::TM_O0 + uint32_t(C::OW) * w, a_tmem + 8u * kk,
+                                bdesc + uint64_t((16 * C::ROW * kk) >> 4), C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+                ptx::mma_commit(bar(C::BAR_VE + s));
+                ptx::mma_commit(bar(C::BAR_PE + 2 * w + (j & 1)));
+                ++v_used;
+                return true;
+            };
+            // The S buffer is shared: slice 0's Q K^T for block j follows the last
+            // slice's read of block j-1, slice 1's follows slice 0's read of block j.
+            for (int j = 0; j < nkb && ok; ++j) {
+                if (j > 0) ok = wait_fast(bar(C::BAR_SE + (n_valid - 1)), (j - 1) & 1, abort_flag);
+                ok = ok && issue_qk(0);
+                if (n_valid == 2) ok = ok && wait_fast(bar(C::BAR_SE + 0), j & 1, abort_flag) && issue_qk(1);
+                if (j > 0)
+                    for (int w = 0; w < n_valid && ok; ++w) ok = issue_pv(w, j - 1);
             }
+            for (int w = 0; w < n_valid && ok; ++w) ok = issue_pv(w, nkb - 1);
             if (!ok) {
                 // Wait for every MMA this thread issued before tensor memory is freed.
                 ptx::mma_commit(bar(C::BAR_DRAIN));
@@ -490,8 +503,8 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int r = lane0 + (lane >> 2) + 8 * (lane & 1);  // query row in the tile == TMEM lane
         if (w < n_valid) {
             const uint32_t lane_base = uint32_t(lane0) << 16;
-            const uint32_t tS = tmem + lane_base + C::TM_S0 + 128u * w;
-            const uint32_t tP = tmem + lane_base + C::TM_P0 + 64u * w;
+            const uint32_t tS = tmem + lane_base + C::TM_S;
+            const uint32_t tP0 = tmem + lane_base + C::TM_P0 + 128u * w;  // + 64 * buffer
             const uint32_t tO = tmem + lane_base + C::TM_O0 + uint32_t(C::OW) * w;
             const float2 l2e2 = make_float2(kLog2e, kLog2e);
             const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
@@ -588,13 +601,19 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 if (!C::SUM_MMA) l = l * alpha + (acc.x + acc.y);
 
-                if (j > 0) {
-                    // P and O of the previous block are in use until its P.V is done; the
-                    // exp pass above overlaps that MMA.
-                    ok = wait_warp(bar(C::BAR_PE + w), (j - 1) & 1, abort_flag);
+                // P buffer j & 1 was last read by the P.V of block j - 2
+                const uint32_t tP = tP0 + 64u * uint32_t(j & 1);
+                if (j >= 2) {
+                    ok = wait_warp(bar(C::BAR_PE + 2 * w + (j & 1)), ((j - 2) >> 1) & 1, abort_flag);
                     if (!ok) break;
                     ptx::tc_fence_after();
-                    if (__any_sync(0xffffffffu, rescale)) {
+                }
+                if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+                    // O holds every block before j once the P.V of block j - 1 is done
+                    ok = wait_warp(bar(C::BAR_PE + 2 * w + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    {
 #pragma unroll
                         for (int dc = 0; dc < C::OW; dc += 16) {  // 8 repeats of 2 columns
                             uint32_t o[8];
@@ -620,10 +639,10 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive_elect(bar(C::BAR_PF + w));
+                ptx::mbar_arrive_elect(bar(C::BAR_PF + 2 * w + (j & 1)));
             }
             // ---------------------------------------------------------- epilogue
-            if (ok) ok = wait_warp(bar(C::BAR_PE + w), (nkb - 1) & 1, abort_flag);
+            if (ok) ok = wait_warp(bar(C::BAR_PE + 2 * w + ((nkb - 1) & 1)), ((nkb - 1) >> 1) & 1, abort_flag);
             if (ok) {
                 ptx::tc_fence_after();
                 const int n = n0 + w;
