@@ -36,7 +36,7 @@ __device__ __noinline__ bool wait_bounded_for(uint32_t bar, uint32_t parity, uin
 // does not complete within kWaitTimeoutNs; returns false at once if another
 // thread of the CTA has already raised the flag (pass abort_flag = nullptr to
 // wait regardless of it, as the drain paths do).
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = ptx::globaltimer_ns();
     while (true) {

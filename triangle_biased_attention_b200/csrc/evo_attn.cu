@@ -121,6 +121,9 @@ int launch_bf16(int dev, const void* Q, const void* K, const void* V, const void
     p.num_qb = int((S + evo::kBM - 1) / evo::kBM);
     p.num_np = int((N + 1) / 2);
     p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
+    p.sqrt_d = float(std::sqrt(double(D)));
+    // the mask (or -inf for keys past S in a ragged last block) enters the score MMA
+    p.aug = (mask != nullptr || S % evo::kBN != 0) ? 1 : 0;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(int64_t(p.num_qb) * H * p.num_np * B), 1, 1);
