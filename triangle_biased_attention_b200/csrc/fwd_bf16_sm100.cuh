@@ -13,14 +13,16 @@
 //    softmax warpgroups.  CTAs are numbered query block fastest, then head,
 //    so the CTAs that share one (n, h) K/V slice, and the four heads that
 //    share each 256 B stretch of a Q/K/V row, run at the same time and hit L2.
-//  * Warp roles (352 threads, 11 warps): warp 0 issues TMA loads (Q once; K
+//  * Warp roles (384 threads, 12 warps): warp 0 issues TMA loads (Q once; K
 //    and bias tiles through rings of mbarrier-tracked stages); warps 1 and 2
 //    serve slice 0 and 1: each loads its slice's V tiles (a ring of its own),
 //    converts them to fp16, turns the mask row into the mask columns of the
 //    score MMA (below) and issues the slice's tcgen05 MMAs from one thread, in
 //    a fixed order that follows the softmax, each step a blocking wait on one
-//    barrier; warps 3-6 and 7-10 are the softmax warpgroups of slice 0 and 1
-//    (warp w reaches tensor-memory lanes 32 * (w % 4) ..).  A softmax thread
+//    barrier; warp 3 has no role; warps 4-7 and 8-11 are the softmax
+//    warpgroups of slice 0 and 1 (warp w reaches tensor-memory lanes
+//    32 * (w % 4) ..).  setmaxnreg moves registers from the first warpgroup
+//    to the softmax warpgroups.  A softmax thread
 //    owns one query row (one tensor-memory lane) and all 128 keys of a block,
 //    so the row maximum needs no shuffle and the bias row is read with 16 B
 //    loads it uses in full.
@@ -85,8 +87,15 @@ struct Bf16Params {
 
 constexpr int kBM = 128;          // query rows per slice tile
 constexpr int kBN = 128;          // keys per block
-constexpr int kThreads = 352;     // producer + 2 slice helpers + 2 softmax warpgroups
-constexpr int kFirstSoftmaxWarp = 3;
+constexpr int kThreads = 384;     // helper warpgroup (producer, 2 slice helpers, 1 idle) + 2 softmax warpgroups
+constexpr int kFirstSoftmaxWarp = 4;
+// Register split (setmaxnreg): the helper warpgroup hands registers to the two
+// softmax warpgroups, which keep a block's 128 scores in registers and need
+// room beside them to overlap independent work.  The split must not exceed
+// the 384 x 168 registers the block is launched with.
+constexpr int kHelperRegs = 120;
+constexpr int kSoftmaxRegs = 192;
+static_assert(128 * kHelperRegs + 256 * kSoftmaxRegs <= 384 * 168, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 12.0f;  // log2 units: p <= 2^12 (fp16 P) between rescales
@@ -292,6 +301,8 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (warp < kFirstSoftmaxWarp) ptx::setmaxnreg_dec<kHelperRegs>();
+    else ptx::setmaxnreg_inc<kSoftmaxRegs>();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -335,7 +346,7 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         }
         __syncwarp();
-    } else if (warp < kFirstSoftmaxWarp) {
+    } else if (warp < 3) {
         // -------------------------------- helper of slice w: V, mask, MMAs
         // Per block j this warp issues Q K^T(j) once the softmax has pulled
         // S(j-1) into registers, writes the mask columns of block j+1, loads
@@ -522,7 +533,7 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         }
         __syncwarp();
-    } else {
+    } else if (warp >= kFirstSoftmaxWarp) {
         // ------------------------------------------------------------ softmax
         const int w = (warp - kFirstSoftmaxWarp) >> 2;  // slice (n0 + w)
         const int quarter = warp & 3;                   // TMEM lanes 32*quarter .. +31

@@ -184,6 +184,16 @@ __device__ __forceinline__ void tmem_ld_wait_x32(uint32_t* r) {
                  : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t* r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : EVO_R8(0)
+                 : "r"(taddr));
+}
+
+// Waits for this thread's outstanding tcgen05.ld (the registers are tied
+// to the wait by reg_fence_* afterwards).
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void tmem_ld_wait_x16(uint32_t* r) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" : EVO_P8(0), EVO_P8(8) : : "memory");
 }
