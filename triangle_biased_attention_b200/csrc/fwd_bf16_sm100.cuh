@@ -270,6 +270,25 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         ptx::mbar_init(bar(C::BAR_DRAIN + 1), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
+        // Thread 0 is also the producer: Q and the first key block's K and bias
+        // tiles go out now, before the CTA-wide setup below (their shared-memory
+        // regions are not touched by it), so that their latency overlaps it.
+        ptx::prefetch_tmap(&tm_q);
+        ptx::prefetch_tmap(&tm_k);
+        if (HAS_PAIR) ptx::prefetch_tmap(&tm_pair);
+        const int bn0 = b * p.N + n0;
+        ptx::mbar_arrive_expect_tx(bar(C::BAR_Q), uint32_t(n_valid * C::TILE));
+        for (int w = 0; w < n_valid; ++w)
+            ptx::tma_load_4d(sb + C::OFF_Q + w * C::TILE, &tm_q, bar(C::BAR_Q), 0, h, q0, bn0 + w);
+        for (int w = 0; w < n_valid; ++w) {  // K stages 0 and 1 are free
+            ptx::mbar_arrive_expect_tx(bar(C::BAR_KF + w), C::TILE);
+            ptx::tma_load_4d(sb + C::OFF_K + w * C::TILE, &tm_k, bar(C::BAR_KF + w), 0, h, 0, bn0 + w);
+        }
+        if (HAS_PAIR) {  // bias stage 0 is free
+            ptx::mbar_arrive_expect_tx(bar(C::BAR_BF), C::BIAS_BYTES);
+            ptx::tma_load_3d(sb + C::OFF_BIAS, &tm_pair, bar(C::BAR_BF), 0, q0, bh);
+            ptx::tma_load_3d(sb + C::OFF_BIAS + C::BIAS_BYTES / 2, &tm_pair, bar(C::BAR_BF), 64, q0, bh);
+        }
     }
     if (warp == 1) {
         // Constant tiles.  The ones tile (D <= 32), the N-continuation of every
@@ -307,16 +326,11 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            ptx::prefetch_tmap(&tm_q);
-            ptx::prefetch_tmap(&tm_k);
-            if (HAS_PAIR) ptx::prefetch_tmap(&tm_pair);
             const int bn0 = b * p.N + n0;
-            ptx::mbar_arrive_expect_tx(bar(C::BAR_Q), uint32_t(n_valid * C::TILE));
-            for (int w = 0; w < n_valid; ++w)
-                ptx::tma_load_4d(sb + C::OFF_Q + w * C::TILE, &tm_q, bar(C::BAR_Q), 0, h, q0, bn0 + w);
-            int k_issued = 0, b_issued = 0;
+            // Q, K(block 0) and bias(block 0) went out with the barrier setup.
+            int k_issued = n_valid, b_issued = HAS_PAIR ? 1 : 0;
             bool ok = true;
-            for (int j = 0; j < nkb && ok; ++j) {
+            for (int j = 1; j < nkb && ok; ++j) {
                 for (int w = 0; w < n_valid && ok; ++w) {
                     const int s = k_issued % C::K_STAGES;
                     const uint32_t ph = (k_issued / C::K_STAGES) & 1;
@@ -681,6 +695,11 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     // start of the block.  p <= 2^12 unless the block raises the
                     // maximum by more than 12; then P is recomputed below.
                     const float2 nm2 = make_float2(-m_used, -m_used);
+                    // The first kHeldChunks chunks of P stay in registers, so that the
+                    // wait for P.V(j-1) (which still reads the P buffer) comes a few
+                    // chunks into the pass, when that P.V has usually finished.
+                    constexpr int kHeldChunks = 3;
+                    uint32_t held[kHeldChunks][8];
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {  // 16 keys -> 8 P columns per store
                         uint32_t pk[8];
@@ -702,9 +721,16 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                             for (int e = 0; e < 4; ++e) pk[4 * q + e] = exp_pair(s, k + 2 * e, nm2, acc);
                         }
-                        if (c == 0) {
+                        if (c < kHeldChunks) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) held[c][e] = pk[e];
+                            continue;
+                        }
+                        if (c == kHeldChunks) {
                             ok = wait_pv();
                             if (!ok) break;
+#pragma unroll
+                            for (int h2 = 0; h2 < kHeldChunks; ++h2) ptx::tmem_st_x8(tP + 8u * h2, held[h2]);
                         }
                         ptx::tmem_st_x8(tP + 8u * c, pk);
                     }
