@@ -88,6 +88,25 @@ BF16_SHAPES = [
 ]
 
 
+# Large pair-bias spikes scattered over several key blocks: rows whose maximum
+# is raised by more than the kernel's lazy-rescale headroom in a later block
+# take its rare recompute path (and rescale O in tensor memory).
+SPIKE_SHAPES = [
+    # B, N, S, H, D, mask, spike value, spike fraction, seed
+    (1, 4, 512, 2, 32, "tail", 24.0, 0.002, 21),
+    (1, 2, 640, 2, 64, "bernoulli", 30.0, 0.001, 22),
+    (1, 3, 384, 1, 16, "tail", -40.0, 0.01, 23),
+]
+
+
+@pytest.mark.parametrize("shape", SPIKE_SHAPES, ids=lambda s: f"S{s[2]}-D{s[4]}-spike{s[6]:+g}")
+def test_bf16_late_maximum_raises(shape):
+    B, N, S, H, D, mask, spike, frac, seed = shape
+    case = W.random_case(B, N, S, H, D, torch.bfloat16, seed=seed, mask=mask, pair=True,
+                         spike_frac=frac, spike=spike)
+    check_full(case, str(shape), strict=False)
+
+
 @pytest.mark.parametrize("shape", BF16_SHAPES, ids=lambda s: "x".join(map(str, s[:5])) + f"-{s[5]}-{s[6]}")
 def test_bf16_random(shape):
     B, N, S, H, D, pair, mask, full, spike = shape

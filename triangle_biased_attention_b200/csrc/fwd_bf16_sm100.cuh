@@ -702,7 +702,8 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     uint32_t held[kHeldChunks][8];
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {  // 16 keys -> 8 P columns per store
-                        uint32_t pk[8];
+                        uint32_t pk_own[8];
+                        uint32_t* pk = c < kHeldChunks ? held[c < kHeldChunks ? c : 0] : pk_own;
 #pragma unroll
                         for (int q = 0; q < 2; ++q) {
                             const int k = 16 * c + 8 * q;
@@ -721,11 +722,7 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                             for (int e = 0; e < 4; ++e) pk[4 * q + e] = exp_pair(s, k + 2 * e, nm2, acc);
                         }
-                        if (c < kHeldChunks) {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) held[c][e] = pk[e];
-                            continue;
-                        }
+                        if (c < kHeldChunks) continue;  // computed straight into held[c]
                         if (c == kHeldChunks) {
                             ok = wait_pv();
                             if (!ok) break;
