@@ -57,19 +57,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uin
     return ok != 0;
 }
 
-// Non-blocking form of mbar_try_wait: tests the phase once, never suspends.
-__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // ----------------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -184,38 +171,11 @@ __device__ __forceinline__ void tmem_ld_wait_x32(uint32_t* r) {
                  : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld_x8(uint32_t taddr, uint32_t* r) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : EVO_R8(0)
-                 : "r"(taddr));
-}
-
-// Waits for this thread's outstanding tcgen05.ld (the registers are tied
-// to the wait by reg_fence_* afterwards).
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
 __device__ __forceinline__ void tmem_ld_wait_x16(uint32_t* r) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" : EVO_P8(0), EVO_P8(8) : : "memory");
 }
 
 __device__ __forceinline__ void reg_fence_x8(uint32_t* r) { asm volatile("" : EVO_P8(0) : : "memory"); }
-
-// Two 16x64b loads of 32 columns each (TMEM columns c0 .. c0+63 of the warp's
-// 16 lanes) and the wait for them, in one statement: the registers are valid
-// when it returns.
-__device__ __forceinline__ void tmem_ld_16x64b_x64_wait(uint32_t taddr, uint32_t* r) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.16x64b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
-        "tcgen05.ld.sync.aligned.16x64b.x32.b32 "
-        "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : EVO_R8(0), EVO_R8(8), EVO_R8(16), EVO_R8(24), EVO_R8(32), EVO_R8(40), EVO_R8(48), EVO_R8(56)
-        : "r"(taddr), "r"(taddr + 64u)
-        : "memory");
-}
 
 // One lane of the (converged) warp arrives on the mbarrier; no branch.
 __device__ __forceinline__ void mbar_arrive_elect(uint32_t bar) {
@@ -229,58 +189,6 @@ __device__ __forceinline__ void mbar_arrive_elect(uint32_t bar) {
 // Orders later uses of 32 more registers after a preceding wait (no instruction).
 __device__ __forceinline__ void reg_fence_x32(uint32_t* r) {
     asm volatile("" : EVO_P8(0), EVO_P8(8), EVO_P8(16), EVO_P8(24) : : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t* r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        EVO_I8(0), EVO_I8(8), EVO_I8(16), EVO_I8(24)
-        : "memory");
-}
-
-// 16-lane shapes: a warp covers 16 TMEM lanes; in .16x64b thread t holds
-// lane (t >> 2) + 8 * (t & 1) of the group and, for repeat i, the 32-bit
-// column 2 * i + ((t >> 1) & 1).  Lanes t and t ^ 2 therefore share a lane.
-__device__ __forceinline__ void tmem_ld_16x64b_x32(uint32_t taddr, uint32_t* r) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.16x64b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : EVO_R8(0), EVO_R8(8), EVO_R8(16), EVO_R8(24)
-        : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_ld_16x64b_x16(uint32_t taddr, uint32_t* r) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.16x64b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : EVO_R8(0), EVO_R8(8)
-        : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_ld_16x64b_x8(uint32_t taddr, uint32_t* r) {
-    asm volatile("tcgen05.ld.sync.aligned.16x64b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : EVO_R8(0)
-                 : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_ld_wait_x8(uint32_t* r) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;" : EVO_P8(0) : : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_16x64b_x16(uint32_t taddr, const uint32_t* r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.16x64b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-        EVO_I8(0), EVO_I8(8)
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_16x64b_x8(uint32_t taddr, const uint32_t* r) {
-    asm volatile("tcgen05.st.sync.aligned.16x64b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), EVO_I8(0)
-                 : "memory");
 }
 
 __device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t* r) {
@@ -339,14 +247,6 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
-}
-
-__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr));
-    return v;
 }
 
 // bf16 pair in one 32-bit word -> two floats (low half is the lower index).
