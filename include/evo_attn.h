@@ -22,9 +22,11 @@
  * side, already transposed).
  *
  * Conventions for every entry point:
- *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *    keeps no reference to them after the call returns and allocates nothing
- *    per call.
+ *  - All tensor pointers are DEVICE pointers owned by the caller, all on one
+ *    device (else EVO_ERR_INVALID_ARG).  The call runs on the device that owns
+ *    Q and leaves the caller's current device as it found it.  The library
+ *    keeps no reference to the pointers after the call returns and allocates
+ *    nothing per call.
  *  - Tensors are dense and contiguous (row-major in the shapes above).
  *  - Calls are asynchronous on `stream` (NULL = the legacy default stream);
  *    the library never synchronises on its own.

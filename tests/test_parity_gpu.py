@@ -166,3 +166,18 @@ def test_zero_sized_call_is_a_noop():
 
 def test_status_is_clear_after_parity_runs():
     assert evo.evo_attn_sync_status() == evo.EVO_OK
+
+
+def test_buffers_on_another_device_are_rejected():
+    """Every buffer must live on Q's device; a host (pinned) buffer is refused
+    before anything is launched, and the caller's current device is kept."""
+    case = W.random_case(1, 2, 128, 1, 32, torch.bfloat16, seed=8, mask="tail", pair=True)
+    dev = torch.device("cuda", 0)
+    q, k, v = (t.to(dev) for t in (case.q, case.k, case.v))
+    o = torch.empty_like(q)
+    lse_host = torch.empty((1, 2, 1, 128), dtype=torch.float32).pin_memory()
+    before = torch.cuda.current_device()
+    st = evo.evo_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), None, None, o.data_ptr(), lse_host.data_ptr(),
+                          1, 2, 128, 1, 32, evo.EVO_DTYPE_BF16, None)
+    assert st == evo.EVO_ERR_INVALID_ARG
+    assert torch.cuda.current_device() == before

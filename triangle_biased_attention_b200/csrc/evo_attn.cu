@@ -51,19 +51,38 @@ bool overlap(const void* a, int64_t abytes, const void* b, int64_t bbytes) {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-// Make this library's runtime use the device that owns `ptr` (the caller's
-// framework may keep its own notion of the current device).
-int select_device_of(const void* ptr) {
+// The device that owns `ptr`, or a negative status if it is not device memory.
+int device_of(const void* ptr) {
     cudaPointerAttributes attr;
     if (cudaPointerGetAttributes(&attr, ptr) != cudaSuccess) {
         cudaGetLastError();
         return EVO_ERR_INVALID_ARG;
     }
     if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return EVO_ERR_INVALID_ARG;
+    return attr.device;
+}
+
+// Makes the device that owns the buffers current for the duration of one
+// call and restores the caller's current device afterwards.
+struct DeviceScope {
+    int prev = -1;
+    bool changed = false;
+    ~DeviceScope() {
+        if (changed) cudaSetDevice(prev);
+    }
+};
+
+int select_device_of(const void* ptr, DeviceScope& scope) {
+    const int dev = device_of(ptr);
+    if (dev < 0) return dev;
     int cur = -1;
     if (cudaGetDevice(&cur) != cudaSuccess) return EVO_ERR_CUDA;
-    if (cur != attr.device && cudaSetDevice(attr.device) != cudaSuccess) return EVO_ERR_CUDA;
-    return attr.device;
+    if (cur != dev) {
+        if (cudaSetDevice(dev) != cudaSuccess) return EVO_ERR_CUDA;
+        scope.prev = cur;
+        scope.changed = true;
+    }
+    return dev;
 }
 
 // Q/K/V/O as a 4-D tensor {D, H, S, B*N}; a box is one (b, n, h) slice's
@@ -191,7 +210,8 @@ __global__ void selftest_timeout_kernel(uint64_t limit_ns, int* result) {
 
 extern "C" EVO_API int evo_attn_selftest_timeout(int64_t limit_ns, int* result, evo_stream_t stream) {
     if (limit_ns <= 0 || limit_ns > 1000000000ll || result == nullptr) return EVO_ERR_INVALID_ARG;
-    const int dev = select_device_of(result);
+    DeviceScope scope;
+    const int dev = select_device_of(result, scope);
     if (dev < 0) return dev;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1, 1, 1);
@@ -253,9 +273,13 @@ extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
             return EVO_ERR_MISALIGNED;
     }
 
-    const int dev = select_device_of(Q);
+    DeviceScope scope;
+    const int dev = select_device_of(Q, scope);
     if (dev < 0) return dev;
     if (dev >= kMaxDevices) return EVO_ERR_UNSUPPORTED_SHAPE;
+    // every buffer must live on Q's device
+    for (const void* ptr : {K, V, static_cast<const void*>(O), static_cast<const void*>(LSE), mask_bias, pair_bias})
+        if (ptr != nullptr && device_of(ptr) != dev) return EVO_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
     if (dtype == EVO_DTYPE_FP32) return launch_f32(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, st);
