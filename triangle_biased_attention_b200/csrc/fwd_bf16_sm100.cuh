@@ -16,10 +16,13 @@
 //  * Warp roles (384 threads, 12 warps): warp 0 issues TMA loads (Q once; K
 //    and bias tiles through rings of mbarrier-tracked stages); warps 1 and 2
 //    serve slice 0 and 1: each loads its slice's V tiles (a ring of its own),
-//    converts them to fp16, turns the mask row into the mask columns of the
-//    score MMA (below) and issues the slice's tcgen05 MMAs from one thread, in
-//    a fixed order that follows the softmax, each step a blocking wait on one
-//    barrier; warp 3 has no role; warps 4-7 and 8-11 are the softmax
+//    turns the mask row into the mask columns of the score MMA (below) and
+//    issues the slice's tcgen05 MMAs from one thread, in a fixed order that
+//    follows the softmax, each step a blocking wait on one barrier; warp 3
+//    converts the V tiles of both slices to fp16, so that no MMA issue waits
+//    behind a V load or its conversion (for D = 64, whose tiles are twice as
+//    large, each helper converts the first half of its own); warps 4-7 and
+//    8-11 are the softmax
 //    warpgroups of slice 0 and 1 (warp w reaches tensor-memory lanes
 //    32 * (w % 4) ..).  setmaxnreg moves registers from the first warpgroup
 //    to the softmax warpgroups.  A softmax thread
@@ -87,14 +90,14 @@ struct Bf16Params {
 
 constexpr int kBM = 128;          // query rows per slice tile
 constexpr int kBN = 128;          // keys per block
-constexpr int kThreads = 384;     // helper warpgroup (producer, 2 slice helpers, 1 idle) + 2 softmax warpgroups
+constexpr int kThreads = 384;     // helper warpgroup (producer, 2 slice helpers, V converter) + 2 softmax warpgroups
 constexpr int kFirstSoftmaxWarp = 4;
 // Register split (setmaxnreg): the helper warpgroup hands registers to the two
 // softmax warpgroups, which keep a block's 128 scores in registers and need
 // room beside them to overlap independent work.  The split must not exceed
 // the 384 x 168 registers the block is launched with.
-constexpr int kHelperRegs = 120;
-constexpr int kSoftmaxRegs = 192;
+constexpr int kHelperRegs = 96;
+constexpr int kSoftmaxRegs = 200;
 static_assert(128 * kHelperRegs + 256 * kSoftmaxRegs <= 384 * 168, "register split");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -115,6 +118,9 @@ struct Bf16Cfg {
     static constexpr int OW = D + (SUM_MMA ? 16 : 0); // O accumulator columns
     static constexpr int K_STAGES = (D <= 32) ? 4 : 2;  // K tiles, block-major then slice
     static constexpr int V_STAGES = (D <= 32) ? 3 : 2;  // V tiles per slice
+    static constexpr int V_CHUNKS = TILE / 16 / 32;     // 16 B chunks per lane in a V tile
+    // chunks per lane the slice's helper converts (warp 3 converts the rest)
+    static constexpr int V_HELPER_CHUNKS = (D == 64) ? V_CHUNKS / 2 : 0;
     static constexpr int AUG_ROW = 32;                // mask columns: 16 bf16 per row
     static constexpr int AUG_TILE = kBM * AUG_ROW;
     static constexpr int M_STAGES = 2;                // mask-column tiles per slice
@@ -137,7 +143,8 @@ struct Bf16Cfg {
     static constexpr int BAR_KE = BAR_KF + K_STAGES;        // K tile consumed
     static constexpr int BAR_VF = BAR_KE + K_STAGES;        // [2][V_STAGES] V tile landed (bf16)
     static constexpr int BAR_VE = BAR_VF + 2 * V_STAGES;    // [2][V_STAGES] V tile consumed
-    static constexpr int BAR_BF = BAR_VE + 2 * V_STAGES;    // [3] bias tile landed
+    static constexpr int BAR_VC = BAR_VE + 2 * V_STAGES;    // [2][V_STAGES] V tile converted to fp16
+    static constexpr int BAR_BF = BAR_VC + 2 * V_STAGES;    // [3] bias tile landed
     static constexpr int BAR_BE = BAR_BF + 3;               // [3] bias tile consumed
     static constexpr int BAR_MF = BAR_BE + 3;               // [2][M_STAGES] mask columns written
     static constexpr int BAR_ME = BAR_MF + 2 * M_STAGES;    // [2][M_STAGES] used by MMA and softmax
@@ -210,6 +217,32 @@ __device__ __forceinline__ uint32_t swz_chunk(int r, int c) {
     return uint32_t(r * ROW) + uint32_t((c ^ sw) << 4);
 }
 
+// 16 B chunks FIRST .. FIRST + COUNT - 1 of every lane (chunk g of lane l is
+// the tile's chunk l + 32 g) of a V tile, bf16 -> fp16 in place (same
+// swizzled positions), by one warp; then the async-proxy fence that makes the
+// generic writes visible to the tensor cores.
+template <int FIRST, int COUNT>
+__device__ __forceinline__ void convert_v_chunks(uint32_t tile, int lane) {
+    static_assert(FIRST % 4 == 0 && COUNT % 4 == 0, "whole groups of four");
+#pragma unroll
+    for (int g = FIRST; g < FIRST + COUNT; g += 4) {
+        uint4 vv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) vv[u] = ptx::ld_shared_v4(tile + uint32_t((lane + 32 * (g + u)) * 16));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            uint4 o;
+            o.x = ptx::pack_f16x2(ptx::bf16lo_to_f32(vv[u].x), ptx::bf16hi_to_f32(vv[u].x));
+            o.y = ptx::pack_f16x2(ptx::bf16lo_to_f32(vv[u].y), ptx::bf16hi_to_f32(vv[u].y));
+            o.z = ptx::pack_f16x2(ptx::bf16lo_to_f32(vv[u].z), ptx::bf16hi_to_f32(vv[u].z));
+            o.w = ptx::pack_f16x2(ptx::bf16lo_to_f32(vv[u].w), ptx::bf16hi_to_f32(vv[u].w));
+            ptx::st_shared_v4(tile + uint32_t((lane + 32 * (g + u)) * 16), o);
+        }
+    }
+    ptx::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+    __syncwarp();
+}
+
 template <int D, bool HAS_PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -251,6 +284,7 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int s = 0; s < 2 * C::V_STAGES; ++s) {
             ptx::mbar_init(bar(C::BAR_VF + s), 1);
             ptx::mbar_init(bar(C::BAR_VE + s), 1);
+            ptx::mbar_init(bar(C::BAR_VC + s), C::V_HELPER_CHUNKS > 0 ? 2 : 1);  // warp 3 (+ helper)
         }
         for (int s = 0; s < 3; ++s) {
             ptx::mbar_init(bar(C::BAR_BF + s), 1);
@@ -360,194 +394,202 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         }
         __syncwarp();
-    } else if (warp < 3) {
-        // -------------------------------- helper of slice w: V, mask, MMAs
-        // Per block j this warp issues Q K^T(j) once the softmax has pulled
-        // S(j-1) into registers, writes the mask columns of block j+1, loads
-        // and converts V, and issues P.V(j-1) once the softmax has written
-        // P(j-1): a fixed order that follows the softmax, each step a blocking
-        // wait on one barrier (no polling).  Lane 0 issues the MMAs.
-        const int w = warp - 1;
-        if (w < n_valid) {
-            const uint16_t* mrow = p.mask != nullptr ? p.mask + (size_t(b) * p.N + n0 + w) * size_t(p.S) : nullptr;
-            float c_run = -INFINITY;
+    } else if (warp < kFirstSoftmaxWarp) {
+        // Both roles of the helper warpgroup sit under the same condition as its
+        // setmaxnreg above; as separate branches of this if-chain the code
+        // generator no longer held them to the smaller register budget and
+        // spilled.
+        if (warp == 3) {
+            // ---------------------------------- V to fp16, both slices
+            // Block by block, slice 0 then slice 1.  A V tile is reloaded only
+            // after its P.V, which waits for this warp's conversion, so this
+            // warp is never a whole ring behind the barrier phases it waits on.
             bool ok = true;
-            // mask values of a block, fetched one block before they are needed:
-            // lane l handles keys l, l+32, l+64, l+96
-            uint32_t raw[4] = {0u, 0u, 0u, 0u};
-            auto fetch = [&](int j) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int key = j * kBN + lane + 32 * k;
-                    raw[k] = (mrow != nullptr && key < p.S) ? uint32_t(mrow[key]) : 0u;
-                }
-            };
-            auto write_mask = [&](int j) -> bool {
-                float v[4];
-                float bmax = -INFINITY;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int key = j * kBN + lane + 32 * k;
-                    v[k] = key < p.S ? __uint_as_float(raw[k] << 16) : -INFINITY;
-                    bmax = fmaxf(bmax, v[k]);
-                }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
-                c_run = fmaxf(c_run, bmax);
-                const float csub = (c_run == -INFINITY) ? 0.f : c_run;  // all -inf so far: keep -inf logits
-                const int stage = j % C::M_STAGES;
-                const int ms = w * C::M_STAGES + stage;
-                if (!wait_warp(bar(C::BAR_ME + ms), ((j / C::M_STAGES) & 1) ^ 1, abort_flag)) return false;
-                const uint32_t tile = sb + C::OFF_KAUG + uint32_t(ms * C::AUG_TILE);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int key = lane + 32 * k;
-                    // (mask - c) * sqrt(D) as hi + mid + lo, three bf16 that sum to the fp32 value
-                    const float x = (v[k] - csub) * p.sqrt_d;
-                    const uint32_t hi = ptx::f32_to_bf16_bits(x);
-                    uint32_t mid = 0, lo = 0;
-                    if (fabsf(x) < INFINITY) {
-                        const float r1 = x - __uint_as_float(hi << 16);
-                        mid = ptx::f32_to_bf16_bits(r1);
-                        lo = ptx::f32_to_bf16_bits(r1 - __uint_as_float(mid << 16));
-                    }
-                    ptx::st_shared_v2(tile + swz_chunk<C::AUG_ROW>(key, 0), hi | (mid << 16), lo);
-                }
-                if (lane == 0) mc_s[ms] = csub;
-                ptx::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(C::BAR_MF + ms));
-                return true;
-            };
-            // This warp loads the slice's V tiles itself (lane 0), V_STAGES ahead,
-            // so that V never waits behind K or the bias in another thread's queue.
-            const int bn = b * p.N + n0 + w;
-            int v_issued = 0;
-            auto load_v = [&](int j) -> bool {
-                const int vs = w * C::V_STAGES + j % C::V_STAGES;
-                // the tile's previous block (j - V_STAGES) must be consumed by its P.V
-                if (!wait_warp(bar(C::BAR_VE + vs), ((j / C::V_STAGES) & 1) ^ 1, abort_flag)) return false;
-                if (lane == 0) {
-                    ptx::mbar_arrive_expect_tx(bar(C::BAR_VF + vs), C::TILE);
-                    ptx::tma_load_4d(sb + C::OFF_V + vs * C::TILE, &tm_v, bar(C::BAR_VF + vs), 0, h, j * kBN, bn);
-                }
-                v_issued = j + 1;
-                return true;
-            };
-            // V tile of block j: bf16 -> fp16 in place, same swizzled positions
-            auto convert_v = [&](int j) -> bool {
-                const int vs = w * C::V_STAGES + j % C::V_STAGES;
-                if (!wait_warp(bar(C::BAR_VF + vs), (j / C::V_STAGES) & 1, abort_flag)) return false;
-                const uint32_t tile = sb + C::OFF_V + uint32_t(vs * C::TILE);
-                constexpr int PER_LANE = C::TILE / 16 / 32;
-#pragma unroll
-                for (int g = 0; g < PER_LANE; g += 4) {
-                    uint4 vv[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) vv[u] = ptx::ld_shared_v4(tile + uint32_t((lane + 32 * (g + u)) * 16));
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        uint4 o;
-                        o.x = ptx::pack_f16x2(ptx::bf16lo_to_f32(vv[u].x), ptx::bf16hi_to_f32(vv[u].x));
-                        o.y = ptx::pack_f16x2(ptx::bf16lo_to_f32(vv[u].y), ptx::bf16hi_to_f32(vv[u].y));
-                        o.z = ptx::pack_f16x2(ptx::bf16lo_to_f32(vv[u].z), ptx::bf16hi_to_f32(vv[u].z));
-                        o.w = ptx::pack_f16x2(ptx::bf16lo_to_f32(vv[u].w), ptx::bf16hi_to_f32(vv[u].w));
-                        ptx::st_shared_v4(tile + uint32_t((lane + 32 * (g + u)) * 16), o);
-                    }
-                }
-                ptx::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
-                __syncwarp();
-                return true;
-            };
-            const uint32_t d_s = tmem + C::TM_S0 + 128u * w;
-            const uint32_t d_o = tmem + C::TM_O0 + uint32_t(C::OW) * w;
-            const uint32_t a_p = tmem + C::TM_P0 + 64u * w;
-            const uint64_t a_q = desc_k_major<C::ROW>(sb + C::OFF_Q + w * C::TILE);
-            bool issued_any = false;
-            auto issue_qk = [&](int j) -> bool {
-                const int ki = j * n_valid + w;  // the producer's K tile order
-                const int ks = ki % C::K_STAGES;
-                if (!wait_warp(bar(C::BAR_KF + ks), (ki / C::K_STAGES) & 1, abort_flag)) return false;
-                if (lane == 0) {
-                    ptx::tc_fence_after();
-                    const uint64_t bd = desc_k_major<C::ROW>(sb + C::OFF_K + ks * C::TILE);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)  // 16 bf16 = 32 B per K step
-                        ptx::mma_ss(d_s, a_q + uint64_t(2 * kk), bd + uint64_t(2 * kk), C::IDESC_QK, kk > 0 ? 1u : 0u);
-                    if (aug) {
-                        const int ms = w * C::M_STAGES + j % C::M_STAGES;
-                        ptx::mma_ss(d_s, desc_k_major<C::AUG_ROW>(sb + C::OFF_QAUG),
-                                    desc_k_major<C::AUG_ROW>(sb + C::OFF_KAUG + ms * C::AUG_TILE), C::IDESC_QK, 1u);
-                        ptx::mma_commit(bar(C::BAR_ME + ms));
-                    }
-                    ptx::mma_commit(bar(C::BAR_KE + ks));
-                    ptx::mma_commit(bar(C::BAR_SF + w));
-                }
-                issued_any = true;
-                __syncwarp();
-                return true;
-            };
-            auto issue_pv = [&](int j) -> bool {
-                // P(j) written by the four softmax warps; V(j) converted by this warp
-                if (!wait_warp(bar(C::BAR_PF + w), j & 1, abort_flag)) return false;
-                if (lane == 0) {
-                    ptx::tc_fence_after();
+            for (int j = 0; j < nkb && ok; ++j) {
+                for (int w = 0; w < n_valid && ok; ++w) {
                     const int vs = w * C::V_STAGES + j % C::V_STAGES;
-                    const uint32_t v_off = uint32_t(C::OFF_V + vs * C::TILE);
-                    // the ones tile continues V along N (D <= 32); unused for D = 64
-                    const uint64_t bd =
-                        desc_mn_major<C::ROW>(sb + v_off, C::SUM_MMA ? uint32_t(C::OFF_ONES) - v_off : uint32_t(C::TILE));
-#pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)  // 16 keys per K step = 16 rows of V
-                        ptx::mma_ts(d_o, a_p + 8u * kk, bd + uint64_t((16 * C::ROW * kk) >> 4), C::IDESC_PV,
-                                    (j > 0 || kk > 0) ? 1u : 0u);
-                    ptx::mma_commit(bar(C::BAR_VE + vs));
-                    ptx::mma_commit(bar(C::BAR_PE + w));
-                }
-                __syncwarp();
-                return true;
-            };
-            if (lane == 0) ptx::prefetch_tmap(&tm_v);
-            // V(0) and V(1) go out first; later V(j+1) is loaded in iteration j,
-            // into the tile that P.V(j+1-V_STAGES) has released.
-            for (int j = 0; j < 2 && j < nkb && ok; ++j) ok = load_v(j);
-            if (aug && ok) {
-                fetch(0);
-                for (int j = 0; j < C::M_STAGES && j < nkb && ok; ++j) {
-                    ok = write_mask(j);
-                    fetch(j + 1);
+                    ok = wait_warp(bar(C::BAR_VF + vs), (j / C::V_STAGES) & 1, abort_flag);
+                    if (!ok) break;
+                    convert_v_chunks<C::V_HELPER_CHUNKS, C::V_CHUNKS - C::V_HELPER_CHUNKS>(
+                        sb + C::OFF_V + uint32_t(vs * C::TILE), lane);
+                    if (lane == 0) ptx::mbar_arrive(bar(C::BAR_VC + vs));
                 }
             }
-            ok = ok && wait_warp(bar(C::BAR_Q), 0, abort_flag);
-            ok = ok && issue_qk(0);
-            ok = ok && convert_v(0);
-            for (int j = 1; j <= nkb && ok; ++j) {
-                if (j < nkb) {
-                    // S(j-1) is in the softmax's registers: Q K^T(j) may overwrite it
-                    ok = wait_warp(bar(C::BAR_SE + w), (j - 1) & 1, abort_flag) && issue_qk(j);
-                    if (ok && aug && j + 1 < nkb) {
-                        ok = write_mask(j + 1);
-                        fetch(j + 2);
+        } else {
+            // -------------------------------- helper of slice w: V, mask, MMAs
+            // Per block j this warp issues Q K^T(j) once the softmax has pulled
+            // S(j-1) into registers, writes the mask columns of block j+1, loads
+            // V, and issues P.V(j-1) once warp 3 has converted V(j-1) and the
+            // softmax has written P(j-1): a fixed order that follows the softmax,
+            // each step a blocking wait on one barrier (no polling).  Lane 0
+            // issues the MMAs.
+            const int w = warp - 1;
+            if (w < n_valid) {
+                const uint16_t* mrow = p.mask != nullptr ? p.mask + (size_t(b) * p.N + n0 + w) * size_t(p.S) : nullptr;
+                float c_run = -INFINITY;
+                bool ok = true;
+                // mask values of a block, fetched one block before they are needed:
+                // lane l handles keys l, l+32, l+64, l+96
+                uint32_t raw[4] = {0u, 0u, 0u, 0u};
+                auto fetch = [&](int j) {
+    #pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int key = j * kBN + lane + 32 * k;
+                        raw[k] = (mrow != nullptr && key < p.S) ? uint32_t(mrow[key]) : 0u;
                     }
-                    if (ok && C::V_STAGES >= 3 && j + 1 < nkb) ok = load_v(j + 1);
-                    ok = ok && convert_v(j);
+                };
+                auto write_mask = [&](int j) -> bool {
+                    float v[4];
+                    float bmax = -INFINITY;
+    #pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int key = j * kBN + lane + 32 * k;
+                        v[k] = key < p.S ? __uint_as_float(raw[k] << 16) : -INFINITY;
+                        bmax = fmaxf(bmax, v[k]);
+                    }
+    #pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
+                    c_run = fmaxf(c_run, bmax);
+                    const float csub = (c_run == -INFINITY) ? 0.f : c_run;  // all -inf so far: keep -inf logits
+                    const int stage = j % C::M_STAGES;
+                    const int ms = w * C::M_STAGES + stage;
+                    if (!wait_warp(bar(C::BAR_ME + ms), ((j / C::M_STAGES) & 1) ^ 1, abort_flag)) return false;
+                    const uint32_t tile = sb + C::OFF_KAUG + uint32_t(ms * C::AUG_TILE);
+    #pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int key = lane + 32 * k;
+                        // (mask - c) * sqrt(D) as hi + mid + lo, three bf16 that sum to the fp32 value
+                        const float x = (v[k] - csub) * p.sqrt_d;
+                        const uint32_t hi = ptx::f32_to_bf16_bits(x);
+                        uint32_t mid = 0, lo = 0;
+                        if (fabsf(x) < INFINITY) {
+                            const float r1 = x - __uint_as_float(hi << 16);
+                            mid = ptx::f32_to_bf16_bits(r1);
+                            lo = ptx::f32_to_bf16_bits(r1 - __uint_as_float(mid << 16));
+                        }
+                        ptx::st_shared_v2(tile + swz_chunk<C::AUG_ROW>(key, 0), hi | (mid << 16), lo);
+                    }
+                    if (lane == 0) mc_s[ms] = csub;
+                    ptx::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(bar(C::BAR_MF + ms));
+                    return true;
+                };
+                // This warp loads the slice's V tiles itself (lane 0), V_STAGES ahead,
+                // so that V never waits behind K or the bias in another thread's queue.
+                const int bn = b * p.N + n0 + w;
+                int v_issued = 0;
+                auto load_v = [&](int j) -> bool {
+                    const int vs = w * C::V_STAGES + j % C::V_STAGES;
+                    // the tile's previous block (j - V_STAGES) must be consumed by its P.V
+                    if (!wait_warp(bar(C::BAR_VE + vs), ((j / C::V_STAGES) & 1) ^ 1, abort_flag)) return false;
+                    if (lane == 0) {
+                        ptx::mbar_arrive_expect_tx(bar(C::BAR_VF + vs), C::TILE);
+                        ptx::tma_load_4d(sb + C::OFF_V + vs * C::TILE, &tm_v, bar(C::BAR_VF + vs), 0, h, j * kBN, bn);
+                    }
+                    v_issued = j + 1;
+                    return true;
+                };
+                // D = 64: the first half of V tile j to fp16 (warp 3 converts the rest)
+                auto convert_v = [&](int j) -> bool {
+                    if (C::V_HELPER_CHUNKS == 0) return true;
+                    const int vs = w * C::V_STAGES + j % C::V_STAGES;
+                    if (!wait_warp(bar(C::BAR_VF + vs), (j / C::V_STAGES) & 1, abort_flag)) return false;
+                    convert_v_chunks<0, C::V_HELPER_CHUNKS>(sb + C::OFF_V + uint32_t(vs * C::TILE), lane);
+                    if (lane == 0) ptx::mbar_arrive(bar(C::BAR_VC + vs));
+                    return true;
+                };
+                const uint32_t d_s = tmem + C::TM_S0 + 128u * w;
+                const uint32_t d_o = tmem + C::TM_O0 + uint32_t(C::OW) * w;
+                const uint32_t a_p = tmem + C::TM_P0 + 64u * w;
+                const uint64_t a_q = desc_k_major<C::ROW>(sb + C::OFF_Q + w * C::TILE);
+                bool issued_any = false;
+                auto issue_qk = [&](int j) -> bool {
+                    const int ki = j * n_valid + w;  // the producer's K tile order
+                    const int ks = ki % C::K_STAGES;
+                    if (!wait_warp(bar(C::BAR_KF + ks), (ki / C::K_STAGES) & 1, abort_flag)) return false;
+                    if (lane == 0) {
+                        ptx::tc_fence_after();
+                        const uint64_t bd = desc_k_major<C::ROW>(sb + C::OFF_K + ks * C::TILE);
+    #pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk)  // 16 bf16 = 32 B per K step
+                            ptx::mma_ss(d_s, a_q + uint64_t(2 * kk), bd + uint64_t(2 * kk), C::IDESC_QK, kk > 0 ? 1u : 0u);
+                        if (aug) {
+                            const int ms = w * C::M_STAGES + j % C::M_STAGES;
+                            ptx::mma_ss(d_s, desc_k_major<C::AUG_ROW>(sb + C::OFF_QAUG),
+                                        desc_k_major<C::AUG_ROW>(sb + C::OFF_KAUG + ms * C::AUG_TILE), C::IDESC_QK, 1u);
+                            ptx::mma_commit(bar(C::BAR_ME + ms));
+                        }
+                        ptx::mma_commit(bar(C::BAR_KE + ks));
+                        ptx::mma_commit(bar(C::BAR_SF + w));
+                    }
+                    issued_any = true;
+                    __syncwarp();
+                    return true;
+                };
+                auto issue_pv = [&](int j) -> bool {
+                    // P(j) written by the four softmax warps; V(j) converted by warp 3 (and this warp)
+                    const int vs = w * C::V_STAGES + j % C::V_STAGES;
+                    if (!wait_warp(bar(C::BAR_VC + vs), (j / C::V_STAGES) & 1, abort_flag)) return false;
+                    if (!wait_warp(bar(C::BAR_PF + w), j & 1, abort_flag)) return false;
+                    if (lane == 0) {
+                        ptx::tc_fence_after();
+                        const uint32_t v_off = uint32_t(C::OFF_V + vs * C::TILE);
+                        // the ones tile continues V along N (D <= 32); unused for D = 64
+                        const uint64_t bd =
+                            desc_mn_major<C::ROW>(sb + v_off, C::SUM_MMA ? uint32_t(C::OFF_ONES) - v_off : uint32_t(C::TILE));
+    #pragma unroll
+                        for (int kk = 0; kk < kBN / 16; ++kk)  // 16 keys per K step = 16 rows of V
+                            ptx::mma_ts(d_o, a_p + 8u * kk, bd + uint64_t((16 * C::ROW * kk) >> 4), C::IDESC_PV,
+                                        (j > 0 || kk > 0) ? 1u : 0u);
+                        ptx::mma_commit(bar(C::BAR_VE + vs));
+                        ptx::mma_commit(bar(C::BAR_PE + w));
+                    }
+                    __syncwarp();
+                    return true;
+                };
+                if (lane == 0) ptx::prefetch_tmap(&tm_v);
+                // V(0) and V(1) go out first; later V(j+1) is loaded in iteration j,
+                // into the tile that P.V(j+1-V_STAGES) has released.
+                for (int j = 0; j < 2 && j < nkb && ok; ++j) ok = load_v(j);
+                if (aug && ok) {
+                    fetch(0);
+                    for (int j = 0; j < C::M_STAGES && j < nkb && ok; ++j) {
+                        ok = write_mask(j);
+                        fetch(j + 1);
+                    }
                 }
-                ok = ok && issue_pv(j - 1);
-                if (ok && C::V_STAGES < 3 && j + 1 < nkb) ok = load_v(j + 1);
-            }
-            if (!ok && lane == 0) {
-                // Wait for every MMA and V copy this warp started before the CTA
-                // frees tensor memory and exits.
-                if (issued_any) {
-                    ptx::mma_commit(bar(C::BAR_DRAIN + w));
-                    wait_bounded(bar(C::BAR_DRAIN + w), 0, nullptr);
+                ok = ok && wait_warp(bar(C::BAR_Q), 0, abort_flag);
+                ok = ok && issue_qk(0);
+                ok = ok && convert_v(0);
+                for (int j = 1; j <= nkb && ok; ++j) {
+                    if (j < nkb) {
+                        // S(j-1) is in the softmax's registers: Q K^T(j) may overwrite it
+                        ok = wait_warp(bar(C::BAR_SE + w), (j - 1) & 1, abort_flag) && issue_qk(j);
+                        if (ok && aug && j + 1 < nkb) {
+                            ok = write_mask(j + 1);
+                            fetch(j + 2);
+                        }
+                        if (ok && C::V_STAGES >= 3 && j + 1 < nkb) ok = load_v(j + 1);
+                        ok = ok && convert_v(j);
+                    }
+                    ok = ok && issue_pv(j - 1);
+                    if (ok && C::V_STAGES < 3 && j + 1 < nkb) ok = load_v(j + 1);
                 }
-                for (int i = (v_issued > C::V_STAGES ? v_issued - C::V_STAGES : 0); i < v_issued; ++i)
-                    wait_bounded(bar(C::BAR_VF + w * C::V_STAGES + i % C::V_STAGES), (i / C::V_STAGES) & 1, nullptr);
+                if (!ok && lane == 0) {
+                    // Wait for every MMA and V copy this warp started before the CTA
+                    // frees tensor memory and exits.
+                    if (issued_any) {
+                        ptx::mma_commit(bar(C::BAR_DRAIN + w));
+                        wait_bounded(bar(C::BAR_DRAIN + w), 0, nullptr);
+                    }
+                    for (int i = (v_issued > C::V_STAGES ? v_issued - C::V_STAGES : 0); i < v_issued; ++i)
+                        wait_bounded(bar(C::BAR_VF + w * C::V_STAGES + i % C::V_STAGES), (i / C::V_STAGES) & 1, nullptr);
+                }
             }
         }
         __syncwarp();
-    } else if (warp >= kFirstSoftmaxWarp) {
+    } else {
         // ------------------------------------------------------------ softmax
         const int w = (warp - kFirstSoftmaxWarp) >> 2;  // slice (n0 + w)
         const int quarter = warp & 3;                   // TMEM lanes 32*quarter .. +31
