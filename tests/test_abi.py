@@ -77,10 +77,23 @@ def test_overlapping_outputs_rejected(lib):
 
 
 def test_bf16_envelope(lib):
-    for d in (8, 24, 48, 128, 256):
+    # A call that passes every argument check reaches the device lookup, which
+    # refuses these made-up pointers as not device memory: on a host without a
+    # GPU that status marks an accepted shape.
+    accepted = call()
+    assert accepted == evo.EVO_ERR_INVALID_ARG
+    # head dims outside {16, 32, 64} up to 128, and pair biases whose rows are
+    # not whole 16-byte units, go to the SIMT kernel
+    for d in (1, 8, 24, 48, 128):
+        assert call(D=d) == accepted
+    assert call(S=60, P=0x800000) == accepted
+    for d in (129, 256):
         assert call(D=d) == evo.EVO_ERR_UNSUPPORTED_SHAPE
-    # a pair bias needs 16-byte rows: S a multiple of 8
-    assert call(S=60, P=0x800000) == evo.EVO_ERR_UNSUPPORTED_SHAPE
+    # the SIMT shapes need 2-byte alignment only
+    assert call(D=48, Q=0x10008, O=0x100002) == accepted
+    assert call(S=60, P=0x800002) == accepted
+    assert call(D=48, Q=0x10001) == evo.EVO_ERR_MISALIGNED
+    # the tensor-core shapes keep the 16-byte rule
     assert call(Q=0x10008) == evo.EVO_ERR_MISALIGNED
     assert call(O=0x100002) == evo.EVO_ERR_MISALIGNED
     assert call(P=0x800008) == evo.EVO_ERR_MISALIGNED

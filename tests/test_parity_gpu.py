@@ -115,6 +115,26 @@ def test_bf16_random(shape):
     check_full(case, str(shape), strict=False)
 
 
+# bf16 shapes outside the tensor-core kernel's envelope: the SIMT kernel with
+# bf16 inputs and output
+BF16_SIMT_SHAPES = [
+    # B, N, S, H, D, pair, mask, fully_masked
+    (1, 3, 70, 2, 128, True, "tail", 1),   # D = 128, pair rows not 16-byte units
+    (2, 2, 45, 3, 8, True, "tail", 0),     # small D, ragged S
+    (1, 2, 130, 2, 48, False, "tail", 0),  # D not a multiple of 16
+    (1, 4, 60, 2, 32, True, "tail", 0),    # D = 32 with S % 8 != 0 and a pair bias
+    (1, 2, 33, 1, 1, True, "zero", 0),     # D = 1
+    (1, 2, 96, 2, 24, False, "neg_inf", 0),
+]
+
+
+@pytest.mark.parametrize("shape", BF16_SIMT_SHAPES, ids=lambda s: "x".join(map(str, s[:5])) + f"-{s[5]}-{s[6]}")
+def test_bf16_simt_shapes(shape):
+    B, N, S, H, D, pair, mask, full = shape
+    case = W.random_case(B, N, S, H, D, torch.bfloat16, seed=5, mask=mask, pair=pair, fully_masked=full)
+    check_full(case, str(shape), strict=False)
+
+
 @pytest.mark.parametrize("seed", [0, 1])
 @pytest.mark.parametrize("name", ["tri_start_384", "msa_row_512"])
 def test_bf16_workload_full(name, seed):

@@ -154,15 +154,18 @@ int launch_bf16(int dev, const void* Q, const void* K, const void* V, const void
     return cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, tp, p) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
 
+// The SIMT kernel: T = float for fp32 inputs, uint16_t (bf16 bits) for the
+// bf16 shapes the tensor-core kernel does not take.
+template <typename T>
 int launch_f32(int dev, const void* Q, const void* K, const void* V, const void* mask, const void* pair, void* O,
                float* LSE, int64_t B, int64_t N, int64_t S, int64_t H, int64_t D, cudaStream_t stream) {
-    evo::F32Params p;
-    p.q = static_cast<const float*>(Q);
-    p.k = static_cast<const float*>(K);
-    p.v = static_cast<const float*>(V);
-    p.mask = static_cast<const float*>(mask);
-    p.pair = static_cast<const float*>(pair);
-    p.out = static_cast<float*>(O);
+    evo::F32Params<T> p;
+    p.q = static_cast<const T*>(Q);
+    p.k = static_cast<const T*>(K);
+    p.v = static_cast<const T*>(V);
+    p.mask = static_cast<const T*>(mask);
+    p.pair = static_cast<const T*>(pair);
+    p.out = static_cast<T*>(O);
     p.lse = LSE;
     p.N = int(N);
     p.S = int(S);
@@ -177,8 +180,8 @@ int launch_f32(int dev, const void* Q, const void* K, const void* V, const void*
     if (!attr_set[dev]) {
         const int max_smem = int(sizeof(float) * (size_t(2 * evo::kF32Keys + evo::kF32Rows) * (evo::kF32MaxD + 1) +
                                                   size_t(evo::kF32Rows) * evo::kF32Keys + evo::kF32Rows));
-        if (cudaFuncSetAttribute(evo::evo_fwd_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(evo::evo_fwd_f32_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 max_smem) != cudaSuccess)
             return EVO_ERR_CUDA;
         attr_set[dev] = true;
     }
@@ -188,7 +191,7 @@ int launch_f32(int dev, const void* Q, const void* K, const void* V, const void*
     cfg.blockDim = dim3(evo::kF32Rows * 32, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    return cudaLaunchKernelEx(&cfg, evo::evo_fwd_f32_kernel, p) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, evo::evo_fwd_f32_kernel<T>, p) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
 
 // One warp initialises an mbarrier that expects one arrival, never arrives,
@@ -249,9 +252,12 @@ extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
 
     if (!aligned(LSE, 4)) return EVO_ERR_MISALIGNED;
     const int64_t int_max = 2147483647;
-    if (dtype == EVO_DTYPE_BF16) {
-        if (D != 16 && D != 32 && D != 64) return EVO_ERR_UNSUPPORTED_SHAPE;
-        if (pair_bias && (S % 8) != 0) return EVO_ERR_UNSUPPORTED_SHAPE;
+    // bf16 runs on the tensor-core kernel for D in {16, 32, 64} when the pair
+    // bias rows are whole 16-byte units (S a multiple of 8); every other bf16
+    // shape with D <= 128 runs on the SIMT kernel
+    const bool tensor_core =
+        dtype == EVO_DTYPE_BF16 && (D == 16 || D == 32 || D == 64) && !(pair_bias && (S % 8) != 0);
+    if (tensor_core) {
         // TMA coordinates are 32-bit; the CTA count (query blocks x heads x
         // n pairs x batch) must fit the grid's x dimension
         int64_t ctas;
@@ -268,8 +274,8 @@ extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
         int64_t blocks;
         if (!mul_ok(bnsh / S, num_qb, &blocks) || blocks > int_max || S > int_max || N > int_max || H > int_max)
             return EVO_ERR_UNSUPPORTED_SHAPE;
-        if (!aligned(Q, 4) || !aligned(K, 4) || !aligned(V, 4) || !aligned(O, 4) ||
-            (pair_bias && !aligned(pair_bias, 4)) || (mask_bias && !aligned(mask_bias, 4)))
+        if (!aligned(Q, es) || !aligned(K, es) || !aligned(V, es) || !aligned(O, es) ||
+            (pair_bias && !aligned(pair_bias, es)) || (mask_bias && !aligned(mask_bias, es)))
             return EVO_ERR_MISALIGNED;
     }
 
@@ -282,7 +288,10 @@ extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
         if (ptr != nullptr && device_of(ptr) != dev) return EVO_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
-    if (dtype == EVO_DTYPE_FP32) return launch_f32(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, st);
+    if (dtype == EVO_DTYPE_FP32)
+        return launch_f32<float>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, st);
+    if (!tensor_core)
+        return launch_f32<uint16_t>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, st);
 
     if (encode_fn() == nullptr) return EVO_ERR_CUDA;
     const bool has_pair = pair_bias != nullptr;

@@ -1,8 +1,12 @@
-// fp32 biased-attention forward: plain FMA arithmetic in fp32 throughout.
+// Biased-attention forward with plain FMA arithmetic in fp32 throughout, for
+// fp32 inputs and for the bf16 shapes the tensor-core kernel does not take.
 //
 // The same operation as the bf16 kernel (DeepSpeed DS4Sci_EvoformerAttention
-// guide, hmyw.cn, sections 4, 5.2 and 5.4) for fp32 inputs, where tensor-core
-// TF32 would not hold a 1e-5 relative error.  One warp owns one query row;
+// guide, hmyw.cn, sections 4, 5.2 and 5.4).  For fp32 inputs it is the whole
+// path, because tensor-core TF32 would not hold a 1e-5 relative error; for
+// bf16 inputs (T = raw bf16 bits) it serves any head dimension up to 128 and
+// pair biases whose rows are not a multiple of 16 bytes, at SIMT speed, with
+// O rounded to bf16 at the end.  One warp owns one query row;
 // K and V blocks of 64 keys are staged in shared memory for the 8 rows of a
 // CTA.  Each lane scores two keys of a block, the warp takes the block max
 // and sum with xor-shuffles, then each lane accumulates its D/32 output
@@ -12,6 +16,8 @@
 
 #include <cstdint>
 
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 
 namespace evo {
@@ -20,13 +26,23 @@ constexpr int kF32Rows = 8;   // query rows (warps) per CTA
 constexpr int kF32Keys = 64;  // keys per shared-memory block
 constexpr int kF32MaxD = 128;
 
+// Element access: fp32 as stored, bf16 as raw bits (exact widening; output
+// rounded to nearest even).
+__device__ __forceinline__ float ld_elem(const float* p, size_t i) { return p[i]; }
+__device__ __forceinline__ float ld_elem(const uint16_t* p, size_t i) { return __uint_as_float(uint32_t(p[i]) << 16); }
+__device__ __forceinline__ void st_elem(float* p, size_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void st_elem(uint16_t* p, size_t i, float x) {
+    p[i] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+template <typename T>  // float, or uint16_t holding bf16
 struct F32Params {
-    const float* q;
-    const float* k;
-    const float* v;
-    const float* mask;  // [B, N, S] or nullptr
-    const float* pair;  // [B, H, S, S] or nullptr
-    float* out;
+    const T* q;
+    const T* k;
+    const T* v;
+    const T* mask;  // [B, N, S] or nullptr
+    const T* pair;  // [B, H, S, S] or nullptr
+    T* out;
     float* lse;
     int N, S, H, D;
     int ld;             // padded smem row (D + 1)
@@ -46,7 +62,8 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-__global__ void __launch_bounds__(kF32Rows * 32) evo_fwd_f32_kernel(const F32Params p) {
+template <typename T>
+__global__ void __launch_bounds__(kF32Rows * 32) evo_fwd_f32_kernel(const F32Params<T> p) {
     extern __shared__ float fsm[];
     float* Ks = fsm;                           // [kF32Keys][ld]
     float* Vs = Ks + kF32Keys * p.ld;          // [kF32Keys][ld]
@@ -68,11 +85,11 @@ __global__ void __launch_bounds__(kF32Rows * 32) evo_fwd_f32_kernel(const F32Par
     const size_t slice_base = size_t(bn) * p.S * row_stride + size_t(h) * D;
 
     // per-(b, n) mask rebase
-    const float* mrow = p.mask ? p.mask + size_t(bn) * p.S : nullptr;
+    const T* mrow = p.mask ? p.mask + size_t(bn) * p.S : nullptr;
     float c = 0.f;
     if (mrow) {
         float mx = -INFINITY;
-        for (int j = threadIdx.x; j < p.S; j += blockDim.x) mx = fmaxf(mx, mrow[j]);
+        for (int j = threadIdx.x; j < p.S; j += blockDim.x) mx = fmaxf(mx, ld_elem(mrow, j));
         mx = warp_max(mx);
         if (lane == 0) red[warp] = mx;
         __syncthreads();
@@ -80,11 +97,11 @@ __global__ void __launch_bounds__(kF32Rows * 32) evo_fwd_f32_kernel(const F32Par
         for (int i = 1; i < kF32Rows; ++i) mx = fmaxf(mx, red[i]);
         c = (mx == -INFINITY) ? 0.f : mx;
     }
-    const float* prow = (p.pair && row < p.S) ? p.pair + (size_t(b) * p.H + h) * size_t(p.S) * p.S + size_t(row) * p.S
-                                               : nullptr;
+    const T* prow = (p.pair && row < p.S) ? p.pair + (size_t(b) * p.H + h) * size_t(p.S) * p.S + size_t(row) * p.S
+                                           : nullptr;
 
     for (int d = lane; d < D; d += 32)
-        Qs[warp * p.ld + d] = row < p.S ? p.q[slice_base + size_t(row) * row_stride + d] : 0.f;
+        Qs[warp * p.ld + d] = row < p.S ? ld_elem(p.q, slice_base + size_t(row) * row_stride + d) : 0.f;
 
     float m = -INFINITY, l = 0.f;
     float o[kF32MaxD / 32] = {0.f, 0.f, 0.f, 0.f};
@@ -94,8 +111,8 @@ __global__ void __launch_bounds__(kF32Rows * 32) evo_fwd_f32_kernel(const F32Par
             const int jj = i / D, d = i - jj * D;
             const int key = kb + jj;
             const size_t off = slice_base + size_t(key) * row_stride + d;
-            Ks[jj * p.ld + d] = key < p.S ? p.k[off] : 0.f;
-            Vs[jj * p.ld + d] = key < p.S ? p.v[off] : 0.f;
+            Ks[jj * p.ld + d] = key < p.S ? ld_elem(p.k, off) : 0.f;
+            Vs[jj * p.ld + d] = key < p.S ? ld_elem(p.v, off) : 0.f;
         }
         __syncthreads();
         float tj[2];
@@ -108,8 +125,8 @@ __global__ void __launch_bounds__(kF32Rows * 32) evo_fwd_f32_kernel(const F32Par
                 float dot = 0.f;
                 for (int d = 0; d < D; ++d) dot = fmaf(Qs[warp * p.ld + d], Ks[jj * p.ld + d], dot);
                 x = dot * p.scale;
-                if (mrow) x += mrow[key] - c;
-                if (prow) x += prow[key];
+                if (mrow) x += ld_elem(mrow, key) - c;
+                if (prow) x += ld_elem(prow, key);
             }
             tj[e] = x;
         }
@@ -139,7 +156,7 @@ __global__ void __launch_bounds__(kF32Rows * 32) evo_fwd_f32_kernel(const F32Par
 #pragma unroll
         for (int i = 0; i < kF32MaxD / 32; ++i) {
             const int d = lane + 32 * i;
-            if (d < D) p.out[slice_base + size_t(row) * row_stride + d] = o[i] * inv_l;
+            if (d < D) st_elem(p.out, slice_base + size_t(row) * row_stride + d, o[i] * inv_l);
         }
         if (lane == 0)
             p.lse[(size_t(bn) * p.H + h) * size_t(p.S) + row] = l > 0.f ? m + logf(l) + c : -INFINITY;
