@@ -9,8 +9,10 @@ seeded inputs).  FLOPs per step are 4*B*N*H*S^2*D.  The kernel-only number
 (``value``) times K back-to-back calls on inputs resident in HBM (1.1 GB of
 inputs, larger than the 126 MB L2, so no flush is needed between steps) with
 CUDA events on the launching stream, bracketed by a barrier and a device
-synchronize, max over ranks.  ``e2e`` times the same call with the inputs
-copied from pinned host memory and O / LSE copied back inside every step.
+synchronize, max over ranks.  ``e2e`` times the host-memory entry point
+(``evo_attn_fwd_host``) on the same workload: every step copies the inputs
+from pinned host memory and O / LSE back, in chunks of n slices whose copies
+overlap the kernels of the neighbouring chunks.
 
 Multi-GPU: the forward pass has no exchange step; each rank runs its own
 replica of the workload on its own GPU (weak scaling, no data-path
@@ -300,20 +302,18 @@ def run_ours(args, rank, world, local):
     ms_per_step = ms_max / args.steps
     value = world * flops * args.steps / (ms_max * 1e-3) / 1e12
 
-    # end to end: pinned host inputs -> device -> kernel -> O, LSE back to pinned host
-    host_in = [t.pin_memory() for t in (case.q, case.k, case.v, case.mask, case.pair) if t is not None]
-    dev_in = [q, k, v] + ([mask] if mask is not None else []) + ([pair] if pair is not None else [])
+    # end to end: pinned host inputs -> device -> kernel -> O, LSE back to
+    # pinned host, through the host-memory entry point (chunked, overlapped)
+    pin = lambda t: None if t is None else t.pin_memory()
+    host_in = [pin(t) for t in (case.q, case.k, case.v, case.mask, case.pair)]
     host_o = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     host_lse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    h2d = sum(t.numel() * t.element_size() for t in host_in if t is not None)
     d2h = host_o.numel() * host_o.element_size() + host_lse.numel() * host_lse.element_size()
+    dev_bufs = (q, k, v, mask, pair, out, lse)
 
     def e2e_step():
-        for h, d in zip(host_in, dev_in):
-            d.copy_(h, non_blocking=True)
-        o_, l_ = evo.evo_attn(q, k, v, mask, pair, out=out, lse=lse, stream=stream)
-        host_o.copy_(o_, non_blocking=True)
-        host_lse.copy_(l_, non_blocking=True)
+        evo.evo_attn_from_host(*host_in, out=host_o, lse=host_lse, device_buffers=dev_bufs, stream=stream)
 
     with torch.cuda.stream(stream):
         for _ in range(2):

@@ -130,6 +130,44 @@ EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
                  int dtype, evo_stream_t stream);
 
 /*
+ * evo_attn_fwd_host — evo_attn_fwd for inputs and outputs in page-locked
+ * HOST memory, with the copies overlapped with the computation.
+ *
+ *   Qh, Kh, Vh, mask_h, pair_h  host inputs, same layouts as evo_attn_fwd
+ *                               (mask_h / pair_h may be NULL).
+ *   Oh, LSEh                    host outputs, same layouts.
+ *   Qd, Kd, Vd, mask_d, pair_d, Od, LSEd
+ *                               device buffers of the full sizes, owned by
+ *                               the caller, used as the device side of the
+ *                               call; mask_d / pair_d are NULL exactly when
+ *                               mask_h / pair_h are.
+ *   B, N, S, H, D, dtype        as for evo_attn_fwd.
+ *   chunk_n                     n slices per chunk (>= 1), or 0 for about
+ *                               eight chunks per batch entry.
+ *   stream                      the call is ordered after the work already
+ *                               on `stream`, and the work on `stream` after
+ *                               it is ordered after its last copy back:
+ *                               synchronise `stream` before reading Oh, LSEh.
+ *
+ * The work is split into chunks of chunk_n n slices (the forward pass is
+ * independent per (b, n); the pair bias of batch entry b is copied once).
+ * For each chunk the library copies its inputs to the device on a copy
+ * stream of its own, runs the kernel on `stream`, and copies O and LSE back
+ * on a second copy stream, so the copy in of one chunk, the kernel of the
+ * previous one and the copy back of the one before run at the same time.
+ * The two copy streams and a few events are created once per device, on
+ * the first call, and kept; concurrent calls on one device are enqueued one
+ * after the other.  Host pointers must be page-locked (cudaHostAlloc or
+ * cudaHostRegister), else EVO_ERR_INVALID_ARG; the device buffers get every
+ * check of evo_attn_fwd, with the same status codes.
+ */
+EVO_API int evo_attn_fwd_host(const void* Qh, const void* Kh, const void* Vh, const void* mask_h,
+                      const void* pair_h, void* Oh, float* LSEh,
+                      void* Qd, void* Kd, void* Vd, void* mask_d, void* pair_d, void* Od, float* LSEd,
+                      int64_t B, int64_t N, int64_t S, int64_t H, int64_t D, int dtype, int64_t chunk_n,
+                      evo_stream_t stream);
+
+/*
  * evo_attn_sync_status — synchronise `stream`, then return and clear the
  * device status word of the current device: EVO_OK, EVO_ERR_TIMEOUT if a
  * kernel gave up waiting since the last call, EVO_ERR_RANGE if a kernel met

@@ -137,3 +137,23 @@ def test_selftest_timeout_rejects_bad_arguments(lib):
     assert evo.evo_attn_selftest_timeout(0, 0x1000, None) == evo.EVO_ERR_INVALID_ARG
     assert evo.evo_attn_selftest_timeout(2 * 10**9, 0x1000, None) == evo.EVO_ERR_INVALID_ARG
     assert evo.evo_attn_selftest_timeout(10**6, None, None) == evo.EVO_ERR_INVALID_ARG
+
+
+def call_host(M=None, P=None, Md=None, Pd=None, chunk_n=0, **kw):
+    """evo_attn_fwd_host with made-up host (0x1...) and device (0x9...) addresses."""
+    d = dict(B=1, N=2, S=64, H=2, D=32, dtype=evo.EVO_DTYPE_BF16)
+    d.update(kw)
+    return evo.evo_attn_fwd_host(0x1000000, 0x2000000, 0x3000000, M, P, 0x4000000, 0x5000000,
+                                 0x91000000, 0x92000000, 0x93000000, Md, Pd, 0x94000000, 0x95000000,
+                                 d["B"], d["N"], d["S"], d["H"], d["D"], d["dtype"], chunk_n, None)
+
+
+def test_host_entry_checks_arguments(lib):
+    assert call_host(B=0) == evo.EVO_OK                       # nothing to do
+    assert call_host(chunk_n=-1) == evo.EVO_ERR_INVALID_ARG
+    assert call_host(M=0x6000000) == evo.EVO_ERR_INVALID_ARG   # host mask without a device mask
+    assert call_host(Pd=0x96000000) == evo.EVO_ERR_INVALID_ARG  # device pair without a host pair
+    assert call_host(D=256) == evo.EVO_ERR_UNSUPPORTED_SHAPE   # the device buffers get evo_attn_fwd's checks
+    assert call_host(dtype=7) == evo.EVO_ERR_UNSUPPORTED_DTYPE
+    # made-up host addresses are not page-locked memory
+    assert call_host() == evo.EVO_ERR_INVALID_ARG

@@ -72,6 +72,8 @@ def load_library():
     vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     lib.evo_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, vp]
     lib.evo_attn_fwd.restype = i32
+    lib.evo_attn_fwd_host.argtypes = [vp] * 14 + [i64, i64, i64, i64, i64, i32, i64, vp]
+    lib.evo_attn_fwd_host.restype = i32
     lib.evo_attn_sync_status.argtypes = [vp]
     lib.evo_attn_sync_status.restype = i32
     lib.evo_attn_strerror.argtypes = [i32]
@@ -88,6 +90,14 @@ def evo_attn_fwd(Q: int, K: int, V: int, mask_bias: Optional[int], pair_bias: Op
                  B: int, N: int, S: int, H: int, D: int, dtype: int, stream: Optional[int]) -> int:
     """The C entry point with raw addresses (ints); returns the status code."""
     return int(load_library().evo_attn_fwd(Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, dtype, stream))
+
+
+def evo_attn_fwd_host(Qh, Kh, Vh, mask_h, pair_h, Oh, LSEh, Qd, Kd, Vd, mask_d, pair_d, Od, LSEd,
+                      B: int, N: int, S: int, H: int, D: int, dtype: int, chunk_n: int,
+                      stream: Optional[int]) -> int:
+    """The C entry point for host-memory inputs, raw addresses; returns the status code."""
+    return int(load_library().evo_attn_fwd_host(Qh, Kh, Vh, mask_h, pair_h, Oh, LSEh, Qd, Kd, Vd, mask_d, pair_d,
+                                                Od, LSEd, B, N, S, H, D, dtype, chunk_n, stream))
 
 
 def evo_attn_sync_status(stream: Optional[int] = None) -> int:
@@ -153,4 +163,56 @@ def evo_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                           stream.cuda_stream)
     if status != EVO_OK:
         raise EvoAttnError(status)
+    return out, lse
+
+
+def evo_attn_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                       mask: Optional[torch.Tensor] = None, pair: Optional[torch.Tensor] = None,
+                       out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                       device_buffers: Optional[Tuple] = None, device=None, chunk_n: int = 0,
+                       stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Biased-attention forward on page-locked host tensors; returns (O, LSE) on the host.
+
+    Same shapes and dtypes as ``evo_attn``, all on the CPU and pinned.  The
+    copies to and from the device overlap the computation (``evo_attn_fwd_host``
+    in include/evo_attn.h).  ``device_buffers`` = (q, k, v, mask, pair, out,
+    lse) device tensors of the full shapes (mask / pair None when absent);
+    allocated on ``device`` (default: the current CUDA device) when not given.
+    Asynchronous on ``stream``: synchronise it before reading the results.
+    """
+    if q.dim() != 5:
+        raise ValueError("q must be [B, N, S, H, D]")
+    B, N, S, H, D = q.shape
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    for name, t, shape in (("k", k, q.shape), ("v", v, q.shape),
+                           ("mask", mask, (B, N, 1, 1, S)), ("pair", pair, (B, 1, H, S, S))):
+        if t is None:
+            continue
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} differs from q dtype {q.dtype}")
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    if lse is None:
+        lse = torch.empty((B, N, H, S), dtype=torch.float32, pin_memory=True)
+    for name, t in (("q", q), ("k", k), ("v", v), ("mask", mask), ("pair", pair), ("out", out), ("lse", lse)):
+        if t is None:
+            continue
+        if t.device.type != "cpu" or not t.is_pinned() or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous page-locked host tensor")
+    if device_buffers is None:
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        like = lambda t: None if t is None else torch.empty(t.shape, dtype=t.dtype, device=dev)
+        device_buffers = (like(q), like(k), like(v), like(mask), like(pair), like(out), like(lse))
+    qd, kd, vd, md, pd, od, ld = device_buffers
+    if stream is None:
+        stream = torch.cuda.current_stream(qd.device)
+    status = evo_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(mask), _ptr(pair),
+                               out.data_ptr(), lse.data_ptr(), qd.data_ptr(), kd.data_ptr(), vd.data_ptr(),
+                               _ptr(md), _ptr(pd), od.data_ptr(), ld.data_ptr(), B, N, S, H, D,
+                               _DTYPES[q.dtype], int(chunk_n), stream.cuda_stream)
+    if status != EVO_OK:
+        raise EvoAttnError(status, "evo_attn_fwd_host")
     return out, lse

@@ -225,9 +225,12 @@ extern "C" EVO_API int evo_attn_selftest_timeout(int64_t limit_ns, int* result, 
                : EVO_ERR_CUDA;
 }
 
-extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V, const void* mask_bias,
-                            const void* pair_bias, void* O, float* LSE, int64_t B, int64_t N, int64_t S, int64_t H,
-                            int64_t D, int dtype, evo_stream_t stream) {
+namespace {
+
+// Every argument check of evo_attn_fwd that needs no CUDA call, in the order
+// the header lists them.  On success *tensor_core says which kernel runs.
+int check_fwd(const void* Q, const void* K, const void* V, const void* mask_bias, const void* pair_bias, void* O,
+              float* LSE, int64_t B, int64_t N, int64_t S, int64_t H, int64_t D, int dtype, bool* tensor_core) {
     if (B < 0 || N < 0 || S < 0 || H < 0 || D < 0) return EVO_ERR_INVALID_ARG;
     if (dtype != EVO_DTYPE_BF16 && dtype != EVO_DTYPE_FP32) return EVO_ERR_UNSUPPORTED_DTYPE;
     if (D == 0) return EVO_ERR_UNSUPPORTED_SHAPE;
@@ -255,9 +258,9 @@ extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
     // bf16 runs on the tensor-core kernel for D in {16, 32, 64} when the pair
     // bias rows are whole 16-byte units (S a multiple of 8); every other bf16
     // shape with D <= 128 runs on the SIMT kernel
-    const bool tensor_core =
+    *tensor_core =
         dtype == EVO_DTYPE_BF16 && (D == 16 || D == 32 || D == 64) && !(pair_bias && (S % 8) != 0);
-    if (tensor_core) {
+    if (*tensor_core) {
         // TMA coordinates are 32-bit; the CTA count (query blocks x heads x
         // n pairs x batch) must fit the grid's x dimension
         int64_t ctas;
@@ -279,15 +282,13 @@ extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
             return EVO_ERR_MISALIGNED;
     }
 
-    DeviceScope scope;
-    const int dev = select_device_of(Q, scope);
-    if (dev < 0) return dev;
-    if (dev >= kMaxDevices) return EVO_ERR_UNSUPPORTED_SHAPE;
-    // every buffer must live on Q's device
-    for (const void* ptr : {K, V, static_cast<const void*>(O), static_cast<const void*>(LSE), mask_bias, pair_bias})
-        if (ptr != nullptr && device_of(ptr) != dev) return EVO_ERR_INVALID_ARG;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    return EVO_OK;
+}
 
+// Launches the forward pass on the current device, `dev`, after check_fwd.
+int launch_fwd(int dev, bool tensor_core, const void* Q, const void* K, const void* V, const void* mask_bias,
+               const void* pair_bias, void* O, float* LSE, int64_t B, int64_t N, int64_t S, int64_t H, int64_t D,
+               int dtype, cudaStream_t st) {
     if (dtype == EVO_DTYPE_FP32)
         return launch_f32<float>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, st);
     if (!tensor_core)
@@ -304,6 +305,73 @@ extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
         default: EVO_LAUNCH(64);
     }
 #undef EVO_LAUNCH
+}
+
+// Every buffer of a call must live on Q's device; makes it current.
+int select_call_device(const void* Q, const void* K, const void* V, const void* O, const void* LSE,
+                       const void* mask_bias, const void* pair_bias, DeviceScope& scope) {
+    const int dev = select_device_of(Q, scope);
+    if (dev < 0) return dev;
+    if (dev >= kMaxDevices) return EVO_ERR_UNSUPPORTED_SHAPE;
+    for (const void* ptr : {K, V, O, LSE, mask_bias, pair_bias})
+        if (ptr != nullptr && device_of(ptr) != dev) return EVO_ERR_INVALID_ARG;
+    return dev;
+}
+
+// Copy streams and events of evo_attn_fwd_host: created once per device on
+// first use, kept for the life of the process, and used under `mu` so that
+// concurrent calls enqueue one after the other.
+struct HostPipe {
+    static constexpr int kRing = 4;  // events reused round-robin across chunks
+    std::mutex mu;
+    bool ready = false;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, done = nullptr;
+    cudaEvent_t in[kRing] = {}, out[kRing] = {};
+};
+HostPipe g_pipes[kMaxDevices];
+
+int init_pipe(HostPipe& hp) {
+    if (hp.ready) return EVO_OK;
+    const unsigned ef = cudaEventDisableTiming;
+    if (cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp.start, ef) != cudaSuccess || cudaEventCreateWithFlags(&hp.done, ef) != cudaSuccess)
+        return EVO_ERR_CUDA;
+    for (int r = 0; r < HostPipe::kRing; ++r)
+        if (cudaEventCreateWithFlags(&hp.in[r], ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&hp.out[r], ef) != cudaSuccess)
+            return EVO_ERR_CUDA;
+    hp.ready = true;
+    return EVO_OK;
+}
+
+bool page_locked(const void* p) {
+    if (p == nullptr) return true;
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return attr.type == cudaMemoryTypeHost;
+}
+
+const char* at(const void* p, int64_t bytes) { return static_cast<const char*>(p) + bytes; }
+char* at(void* p, int64_t bytes) { return static_cast<char*>(p) + bytes; }
+
+}  // namespace
+
+extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V, const void* mask_bias,
+                            const void* pair_bias, void* O, float* LSE, int64_t B, int64_t N, int64_t S, int64_t H,
+                            int64_t D, int dtype, evo_stream_t stream) {
+    bool tensor_core = false;
+    const int st = check_fwd(Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, dtype, &tensor_core);
+    if (st != EVO_OK || B == 0 || N == 0 || S == 0 || H == 0) return st;
+    DeviceScope scope;
+    const int dev = select_call_device(Q, K, V, O, LSE, mask_bias, pair_bias, scope);
+    if (dev < 0) return dev;
+    return launch_fwd(dev, tensor_core, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, dtype,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" EVO_API int evo_attn_sync_status(evo_stream_t stream) {
@@ -338,3 +406,93 @@ extern "C" EVO_API const char* evo_attn_strerror(int status) {
 }
 
 extern "C" EVO_API int evo_attn_version(void) { return 100; }
+
+extern "C" EVO_API int evo_attn_fwd_host(const void* Qh, const void* Kh, const void* Vh, const void* mask_h,
+                                 const void* pair_h, void* Oh, float* LSEh, void* Qd, void* Kd, void* Vd,
+                                 void* mask_d, void* pair_d, void* Od, float* LSEd, int64_t B, int64_t N,
+                                 int64_t S, int64_t H, int64_t D, int dtype, int64_t chunk_n,
+                                 evo_stream_t stream) {
+    // the device buffers get every check of evo_attn_fwd
+    bool tensor_core = false;
+    int st = check_fwd(Qd, Kd, Vd, mask_d, pair_d, Od, LSEd, B, N, S, H, D, dtype, &tensor_core);
+    if (st != EVO_OK) return st;
+    if (chunk_n < 0) return EVO_ERR_INVALID_ARG;
+    if ((mask_h == nullptr) != (mask_d == nullptr) || (pair_h == nullptr) != (pair_d == nullptr))
+        return EVO_ERR_INVALID_ARG;
+    if (B == 0 || N == 0 || S == 0 || H == 0) return EVO_OK;
+    if (!Qh || !Kh || !Vh || !Oh || !LSEh) return EVO_ERR_INVALID_ARG;
+    const int64_t es = dtype == EVO_DTYPE_BF16 ? 2 : 4;
+    // sizes fit int64: check_fwd multiplied them out already
+    const int64_t row = S * H * D * es;  // bytes of one (b, n) slice of Q, K, V or O
+    const int64_t mrow = S * es, lrow = H * S * 4, prow = H * S * S * es;
+    const int64_t qkv_bytes = B * N * row, lse_bytes = B * N * lrow;
+    // host outputs must not overlap each other or any host input
+    const void* ins[5] = {Qh, Kh, Vh, mask_h, pair_h};
+    const int64_t in_bytes[5] = {qkv_bytes, qkv_bytes, qkv_bytes, B * N * mrow, B * prow};
+    if (overlap(Oh, qkv_bytes, LSEh, lse_bytes)) return EVO_ERR_INVALID_ARG;
+    for (int i = 0; i < 5; ++i)
+        if (overlap(Oh, qkv_bytes, ins[i], in_bytes[i]) || overlap(LSEh, lse_bytes, ins[i], in_bytes[i]))
+            return EVO_ERR_INVALID_ARG;
+    for (const void* p : {Qh, Kh, Vh, mask_h, pair_h, static_cast<const void*>(Oh), static_cast<const void*>(LSEh)})
+        if (!page_locked(p)) return EVO_ERR_INVALID_ARG;
+
+    DeviceScope scope;
+    const int dev = select_call_device(Qd, Kd, Vd, Od, LSEd, mask_d, pair_d, scope);
+    if (dev < 0) return dev;
+    HostPipe& hp = g_pipes[dev];
+    std::lock_guard<std::mutex> lock(hp.mu);
+    if (init_pipe(hp) != EVO_OK) return EVO_ERR_CUDA;
+
+    // chunks of an even number of n slices (the tensor-core kernel pairs
+    // them), about eight per batch entry by default
+    int64_t cn = chunk_n > 0 ? chunk_n : 2 * ((N + 15) / 16);
+    if (cn > N) cn = N;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const cudaMemcpyKind h2d = cudaMemcpyHostToDevice, d2h = cudaMemcpyDeviceToHost;
+    // the copies start after the work already on the caller's stream
+    if (cudaEventRecord(hp.start, cs) != cudaSuccess || cudaStreamWaitEvent(hp.h2d, hp.start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(hp.d2h, hp.start, 0) != cudaSuccess)
+        return EVO_ERR_CUDA;
+    int64_t i = 0;
+    for (int64_t b = 0; b < B && st == EVO_OK; ++b) {
+        if (pair_h && cudaMemcpyAsync(at(pair_d, b * prow), at(pair_h, b * prow), prow, h2d, hp.h2d) != cudaSuccess) {
+            st = EVO_ERR_CUDA;
+            break;
+        }
+        for (int64_t n0 = 0; n0 < N; n0 += cn, ++i) {
+            const int64_t nn = (N - n0) < cn ? (N - n0) : cn;
+            const int64_t bn0 = b * N + n0;
+            const int r = int(i % HostPipe::kRing);
+            bool ok = cudaMemcpyAsync(at(Qd, bn0 * row), at(Qh, bn0 * row), nn * row, h2d, hp.h2d) == cudaSuccess &&
+                      cudaMemcpyAsync(at(Kd, bn0 * row), at(Kh, bn0 * row), nn * row, h2d, hp.h2d) == cudaSuccess &&
+                      cudaMemcpyAsync(at(Vd, bn0 * row), at(Vh, bn0 * row), nn * row, h2d, hp.h2d) == cudaSuccess &&
+                      (!mask_h ||
+                       cudaMemcpyAsync(at(mask_d, bn0 * mrow), at(mask_h, bn0 * mrow), nn * mrow, h2d, hp.h2d) ==
+                           cudaSuccess) &&
+                      cudaEventRecord(hp.in[r], hp.h2d) == cudaSuccess &&
+                      cudaStreamWaitEvent(cs, hp.in[r], 0) == cudaSuccess;
+            if (!ok) {
+                st = EVO_ERR_CUDA;
+                break;
+            }
+            st = launch_fwd(dev, tensor_core, at(Qd, bn0 * row), at(Kd, bn0 * row), at(Vd, bn0 * row),
+                            mask_d ? at(mask_d, bn0 * mrow) : nullptr, pair_d ? at(pair_d, b * prow) : nullptr,
+                            at(Od, bn0 * row), reinterpret_cast<float*>(at(LSEd, bn0 * lrow)), 1, nn, S, H, D,
+                            dtype, cs);
+            if (st != EVO_OK) break;
+            ok = cudaEventRecord(hp.out[r], cs) == cudaSuccess && cudaStreamWaitEvent(hp.d2h, hp.out[r], 0) == cudaSuccess &&
+                 cudaMemcpyAsync(at(Oh, bn0 * row), at(Od, bn0 * row), nn * row, d2h, hp.d2h) == cudaSuccess &&
+                 cudaMemcpyAsync(at(LSEh, bn0 * lrow), at(LSEd, bn0 * lrow), nn * lrow, d2h, hp.d2h) == cudaSuccess;
+            if (!ok) {
+                st = EVO_ERR_CUDA;
+                break;
+            }
+        }
+    }
+    // the call ends on the caller's stream after the last copy back, on
+    // error paths too, so that nothing of it is left running unordered
+    if (cudaEventRecord(hp.done, hp.d2h) != cudaSuccess || cudaEventRecord(hp.in[0], hp.h2d) != cudaSuccess ||
+        cudaStreamWaitEvent(cs, hp.done, 0) != cudaSuccess || cudaStreamWaitEvent(cs, hp.in[0], 0) != cudaSuccess)
+        return EVO_ERR_CUDA;
+    return st;
+}
