@@ -126,6 +126,17 @@ def test_python_wrapper_validates_before_calling():
         evo.evo_attn(q.double(), q.double(), q.double())
 
 
+def test_host_wrapper_validates_before_calling():
+    import torch
+    q = torch.zeros(1, 2, 8, 1, 16)
+    with pytest.raises(ValueError, match="page-locked"):
+        evo.evo_attn_from_host(q, q, q)           # pageable host tensors are refused
+    with pytest.raises(ValueError):
+        evo.evo_attn_from_host(q, q[:, :1], q)    # shape mismatch
+    with pytest.raises(TypeError):
+        evo.evo_attn_from_host(q.double(), q.double(), q.double())
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(evo, "_lib", None)
     monkeypatch.setattr(evo, "_LIB_PATH", str(tmp_path / "absent.so"))

@@ -193,15 +193,16 @@ def evo_attn_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
         if t.dtype != q.dtype:
             raise TypeError(f"{name} dtype {t.dtype} differs from q dtype {q.dtype}")
+    def host_ok(name, t):
+        if t is not None and (t.device.type != "cpu" or not t.is_contiguous() or not t.is_pinned()):
+            raise ValueError(f"{name} must be a contiguous page-locked host tensor")
+
+    for name, t in (("q", q), ("k", k), ("v", v), ("mask", mask), ("pair", pair), ("out", out), ("lse", lse)):
+        host_ok(name, t)
     if out is None:
         out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
     if lse is None:
         lse = torch.empty((B, N, H, S), dtype=torch.float32, pin_memory=True)
-    for name, t in (("q", q), ("k", k), ("v", v), ("mask", mask), ("pair", pair), ("out", out), ("lse", lse)):
-        if t is None:
-            continue
-        if t.device.type != "cpu" or not t.is_pinned() or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous page-locked host tensor")
     if device_buffers is None:
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
         like = lambda t: None if t is None else torch.empty(t.shape, dtype=t.dtype, device=dev)
