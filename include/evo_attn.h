@@ -147,7 +147,10 @@ EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
  *   stream                      the call is ordered after the work already
  *                               on `stream`, and the work on `stream` after
  *                               it is ordered after its last copy back:
- *                               synchronise `stream` before reading Oh, LSEh.
+ *                               synchronise `stream` before reading Oh, LSEh,
+ *                               and keep every host and device buffer of the
+ *                               call allocated and unchanged until then (as
+ *                               with cudaMemcpyAsync: the copies run later).
  *
  * The work is split into chunks of chunk_n n slices (the forward pass is
  * independent per (b, n); the pair bias of batch entry b is copied once).

@@ -32,8 +32,8 @@ def on_device(case):
 
 
 def from_host(case, chunk_n, stream=None):
-    o, lse = evo.evo_attn_from_host(pinned(case.q), pinned(case.k), pinned(case.v), pinned(case.mask),
-                                    pinned(case.pair), device="cuda:0", chunk_n=chunk_n, stream=stream)
+    hin = [pinned(getattr(case, n)) for n in ("q", "k", "v", "mask", "pair")]
+    o, lse = evo.evo_attn_from_host(*hin, device="cuda:0", chunk_n=chunk_n, stream=stream)
     if stream is None:
         torch.cuda.current_stream(0).synchronize()
     else:
@@ -79,10 +79,13 @@ def test_back_to_back_calls_reuse_device_buffers():
     like = lambda t: torch.empty(t.shape, dtype=t.dtype, device=dev)
     bufs = (like(a.q), like(a.k), like(a.v), like(a.mask), like(a.pair), like(a.q),
             torch.empty((1, 8, 2, 256), dtype=torch.float32, device=dev))
-    outs = []
+    outs, host_inputs = [], []
     for c in (a, b):
-        outs.append(evo.evo_attn_from_host(pinned(c.q), pinned(c.k), pinned(c.v), pinned(c.mask), pinned(c.pair),
-                                           device_buffers=bufs, chunk_n=2))
+        # the pinned inputs stay referenced until the synchronize below: the
+        # copies run after the call returns
+        hin = [pinned(getattr(c, n)) for n in ("q", "k", "v", "mask", "pair")]
+        host_inputs.append(hin)
+        outs.append(evo.evo_attn_from_host(*hin, device_buffers=bufs, chunk_n=2))
     torch.cuda.current_stream(0).synchronize()
     for c, (o, lse) in zip((a, b), outs):
         o_ref, l_ref = on_device(c)

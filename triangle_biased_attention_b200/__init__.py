@@ -178,7 +178,11 @@ def evo_attn_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     in include/evo_attn.h).  ``device_buffers`` = (q, k, v, mask, pair, out,
     lse) device tensors of the full shapes (mask / pair None when absent);
     allocated on ``device`` (default: the current CUDA device) when not given.
-    Asynchronous on ``stream``: synchronise it before reading the results.
+    Asynchronous on ``stream``: synchronise it before reading the results, and
+    keep the host inputs unchanged until then.  The returned O holds
+    references to the inputs and device buffers, so that they are not freed
+    (and their page-locked blocks not handed out again by PyTorch's host
+    allocator, which does not see the library's copies) while O is alive.
     """
     if q.dim() != 5:
         raise ValueError("q must be [B, N, S, H, D]")
@@ -216,4 +220,5 @@ def evo_attn_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                _DTYPES[q.dtype], int(chunk_n), stream.cuda_stream)
     if status != EVO_OK:
         raise EvoAttnError(status, "evo_attn_fwd_host")
+    out._evo_keepalive = (q, k, v, mask, pair, device_buffers)
     return out, lse

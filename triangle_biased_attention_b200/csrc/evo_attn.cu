@@ -72,6 +72,16 @@ struct DeviceScope {
     }
 };
 
+// Relaxed stream-capture mode for this thread during one call, so that the
+// call's host-side queries (pointer attributes, function attributes, the
+// driver entry point) are allowed while the caller captures a CUDA graph;
+// the launches and copies themselves are captured as usual.
+struct RelaxedCapture {
+    cudaStreamCaptureMode mode = cudaStreamCaptureModeRelaxed;
+    RelaxedCapture() { cudaThreadExchangeStreamCaptureMode(&mode); }
+    ~RelaxedCapture() { cudaThreadExchangeStreamCaptureMode(&mode); }
+};
+
 int select_device_of(const void* ptr, DeviceScope& scope) {
     const int dev = device_of(ptr);
     if (dev < 0) return dev;
@@ -367,6 +377,7 @@ extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
     bool tensor_core = false;
     const int st = check_fwd(Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, dtype, &tensor_core);
     if (st != EVO_OK || B == 0 || N == 0 || S == 0 || H == 0) return st;
+    RelaxedCapture relaxed;
     DeviceScope scope;
     const int dev = select_call_device(Q, K, V, O, LSE, mask_bias, pair_bias, scope);
     if (dev < 0) return dev;
@@ -421,6 +432,7 @@ extern "C" EVO_API int evo_attn_fwd_host(const void* Qh, const void* Kh, const v
         return EVO_ERR_INVALID_ARG;
     if (B == 0 || N == 0 || S == 0 || H == 0) return EVO_OK;
     if (!Qh || !Kh || !Vh || !Oh || !LSEh) return EVO_ERR_INVALID_ARG;
+    RelaxedCapture relaxed;
     const int64_t es = dtype == EVO_DTYPE_BF16 ? 2 : 4;
     // sizes fit int64: check_fwd multiplied them out already
     const int64_t row = S * H * D * es;  // bytes of one (b, n) slice of Q, K, V or O
