@@ -198,6 +198,18 @@ def time_oracle(case, slices_per_step: int, steps: int, warmup: int, seed: int):
     return sum(per_step) / len(per_step), flops_slice * slices_per_step, cores
 
 
+def cpu_model() -> str:
+    """The host CPU's model name and logical CPU count, from /proc/cpuinfo."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return f"{line.split(':', 1)[1].strip()} ({os.cpu_count()} logical CPUs)"
+    except OSError:
+        pass
+    return f"unknown ({os.cpu_count()} logical CPUs)"
+
+
 def cpu_baseline(case, args, target_s: float = 10.0):
     """The oracle on random (b, n, h) slices of the workload, in chunks of
     4 slices per host core, until about `target_s` seconds have been spent."""
@@ -214,6 +226,7 @@ def cpu_baseline(case, args, target_s: float = 10.0):
         n_slices += chunk
         seed += 1
     return {"value": done_flops / done_sec / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "cpu": cpu_model(), "nproc": os.cpu_count(),
             "sample": f"{n_slices} random (b,n,h) slices of {args.workload} ({done_flops / 1e9:.0f} GFLOP "
                       f"in {done_sec:.1f} s, float64 C, OpenMP)"}
 
@@ -236,6 +249,7 @@ def run_reference(args, rank, world):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64)",
         "config": workload_config(wl), "impl": "reference",
         "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "cpu": cpu_model(), "nproc": os.cpu_count(),
                          "sample": f"{slices} random (b,n,h) slices of {args.workload} per step"},
         "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

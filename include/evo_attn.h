@@ -172,10 +172,13 @@ EVO_API int evo_attn_fwd_host(const void* Qh, const void* Kh, const void* Vh, co
 
 /*
  * evo_attn_sync_status — synchronise `stream`, then return and clear the
- * device status word of the current device: EVO_OK, EVO_ERR_TIMEOUT if a
- * kernel gave up waiting since the last call, EVO_ERR_RANGE if a kernel met
- * an out-of-range input, or EVO_ERR_CUDA if the stream itself reports an
- * error.  The first error recorded since the last call is the one returned.
+ * device status word of the stream's device (for the legacy default stream,
+ * NULL: the current device), whichever device is current when it is called;
+ * the caller's current device is left as it was.  Returns EVO_OK,
+ * EVO_ERR_TIMEOUT if a kernel on that device gave up waiting since the last
+ * call, EVO_ERR_RANGE if a kernel met an out-of-range input, or EVO_ERR_CUDA
+ * if the stream itself reports an error.  The first error recorded since the
+ * last call is the one returned.
  */
 EVO_API int evo_attn_sync_status(evo_stream_t stream);
 

@@ -214,6 +214,13 @@ def evo_attn_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     qd, kd, vd, md, pd, od, ld = device_buffers
     if stream is None:
         stream = torch.cuda.current_stream(qd.device)
+    # The copies and kernels run on `stream` (and on the library's copy
+    # streams, which `stream` waits for before the call ends): tell PyTorch's
+    # allocator, so that a buffer dropped early is not handed out again on
+    # its allocation stream while the call still uses it.
+    for t in device_buffers:
+        if t is not None:
+            t.record_stream(stream)
     status = evo_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(mask), _ptr(pair),
                                out.data_ptr(), lse.data_ptr(), qd.data_ptr(), kd.data_ptr(), vd.data_ptr(),
                                _ptr(md), _ptr(pd), od.data_ptr(), ld.data_ptr(), B, N, S, H, D,

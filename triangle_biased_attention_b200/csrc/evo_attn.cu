@@ -28,6 +28,23 @@ using evo::Bf16Cfg;
 
 constexpr int kMaxDevices = 64;
 
+// Sets a kernel's dynamic shared-memory limit once per device.  Calls from
+// several host threads may race on the first use; a mutex orders them and
+// the flag is only set once the attribute call has succeeded.
+struct AttrOnce {
+    std::mutex mu;
+    bool done[kMaxDevices] = {};
+    template <typename K>
+    bool ensure(int dev, K kernel, int smem_bytes) {
+        std::lock_guard<std::mutex> lock(mu);
+        if (done[dev]) return true;
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
+            return false;
+        done[dev] = true;
+        return true;
+    }
+};
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -126,12 +143,8 @@ int launch_bf16(int dev, const void* Q, const void* K, const void* V, const void
                 float* LSE, int64_t B, int64_t N, int64_t S, int64_t H, cudaStream_t stream) {
     using C = Bf16Cfg<D, HAS_PAIR>;
     auto kernel = evo::evo_fwd_bf16_kernel<D, HAS_PAIR>;
-    static bool attr_set[kMaxDevices] = {};
-    if (!attr_set[dev]) {
-        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
-            return EVO_ERR_CUDA;
-        attr_set[dev] = true;
-    }
+    static AttrOnce attr;
+    if (!attr.ensure(dev, kernel, C::SMEM_BYTES)) return EVO_ERR_CUDA;
     CUtensorMap tq, tk, tv, tp;
     std::memset(&tp, 0, sizeof(tp));
     if (!encode_qkv(&tq, Q, B * N, S, H, D) || !encode_qkv(&tk, K, B * N, S, H, D) ||
@@ -186,15 +199,10 @@ int launch_f32(int dev, const void* Q, const void* K, const void* V, const void*
     p.scale = float(1.0 / std::sqrt(double(D)));
     const size_t smem = sizeof(float) * (size_t(2 * evo::kF32Keys + evo::kF32Rows) * p.ld +
                                          size_t(evo::kF32Rows) * evo::kF32Keys + evo::kF32Rows);
-    static bool attr_set[kMaxDevices] = {};
-    if (!attr_set[dev]) {
-        const int max_smem = int(sizeof(float) * (size_t(2 * evo::kF32Keys + evo::kF32Rows) * (evo::kF32MaxD + 1) +
-                                                  size_t(evo::kF32Rows) * evo::kF32Keys + evo::kF32Rows));
-        if (cudaFuncSetAttribute(evo::evo_fwd_f32_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 max_smem) != cudaSuccess)
-            return EVO_ERR_CUDA;
-        attr_set[dev] = true;
-    }
+    static AttrOnce attr;
+    const int max_smem = int(sizeof(float) * (size_t(2 * evo::kF32Keys + evo::kF32Rows) * (evo::kF32MaxD + 1) +
+                                              size_t(evo::kF32Rows) * evo::kF32Keys + evo::kF32Rows));
+    if (!attr.ensure(dev, evo::evo_fwd_f32_kernel<T>, max_smem)) return EVO_ERR_CUDA;
     const long long blocks = (long long)B * N * H * p.num_qb;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(blocks), 1, 1);
@@ -387,6 +395,18 @@ extern "C" EVO_API int evo_attn_fwd(const void* Q, const void* K, const void* V,
 
 extern "C" EVO_API int evo_attn_sync_status(evo_stream_t stream) {
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // The status word read is the one on the stream's device (for the legacy
+    // default stream: the current device), whichever device is current.
+    int dev = -1;
+    if (cudaStreamGetDevice(st, &dev) != cudaSuccess) return EVO_ERR_CUDA;
+    DeviceScope scope;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return EVO_ERR_CUDA;
+    if (cur != dev) {
+        if (cudaSetDevice(dev) != cudaSuccess) return EVO_ERR_CUDA;
+        scope.prev = cur;
+        scope.changed = true;
+    }
     if (cudaStreamSynchronize(st) != cudaSuccess) return EVO_ERR_CUDA;
     int v = 0;
     if (cudaMemcpyFromSymbolAsync(&v, evo::g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
