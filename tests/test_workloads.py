@@ -58,15 +58,14 @@ def test_sample_slices():
     assert all((0, n, h) in s for n in (3, 9) for h in range(8))
 
 
-def test_rne_bf16_matches_round_to_nearest_even():
-    """The parity check's output-rounding model: nearest bf16, ties to even."""
-    from tests.parity import rne_bf16
-    x = np.array([1.0, 1.0 + 2**-8, 1.0 + 3 * 2**-8, 4.0 + 2**-6 * 0.999, -4.33, 0.5])
-    # 1 + 2^-8 is a tie between 1 and 1 + 2^-7: even significand wins (1.0);
-    # 1 + 3*2^-8 ties between 1 + 2^-7 and 1 + 2^-6: even is 1 + 2^-6
-    want = np.array([1.0, 1.0, 1.0 + 2**-6, 4.0, -4.34375, 0.5])
-    assert np.array_equal(rne_bf16(x), want)
-    # never further than half a bf16 spacing from the input
-    r = np.random.default_rng(0).standard_normal(1000) * 8
-    half = np.exp2(np.floor(np.log2(np.abs(r))) - 8)
-    assert np.all(np.abs(rne_bf16(r) - r) <= half)
+def test_half_spacing_bounds_bf16_rounding():
+    """Every fp32 value lies within half_spacing_bf16(its bf16 rounding) of
+    that rounding: the bound the parity check removes from |dO|."""
+    from tests.parity import half_spacing_bf16
+    assert np.allclose(half_spacing_bf16(np.array([1.0, 1.5, 2.0, 7.9, -4.0])), [2**-8, 2**-8, 2**-7, 2**-6, 2**-6])
+    r = torch.from_numpy(np.random.default_rng(0).standard_normal(200000).astype(np.float32) * 8)
+    rb = r.to(torch.bfloat16).double().numpy()
+    assert np.all(np.abs(rb - r.double().numpy()) <= half_spacing_bf16(rb))
+    # ties go to the even significand: 1 + 2^-8 -> 1, 1 + 3*2^-8 -> 1 + 2^-6
+    t = torch.tensor([1.0 + 2**-8, 1.0 + 3 * 2**-8], dtype=torch.float32).to(torch.bfloat16).double()
+    assert t.tolist() == [1.0, 1.0 + 2**-6]
