@@ -20,6 +20,7 @@
 #include "evo_attn.h"
 #include "common.cuh"
 #include "fwd_bf16_sm100.cuh"
+#include "fwd_tri_sm100.cuh"
 #include "fwd_f32.cuh"
 
 namespace {
@@ -177,6 +178,50 @@ int launch_bf16(int dev, const void* Q, const void* K, const void* V, const void
     return cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, tp, p) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
 
+// The three-slice persistent kernel (head dims 16 and 32): one CTA per SM,
+// each walking the tiles (query block, head, n triple, batch) with a stride
+// of the grid size.
+template <int D, bool HAS_PAIR>
+int launch_tri(int dev, const void* Q, const void* K, const void* V, const void* mask, const void* pair, void* O,
+               float* LSE, int64_t B, int64_t N, int64_t S, int64_t H, cudaStream_t stream) {
+    using C = evo::TriCfg<D, HAS_PAIR>;
+    auto kernel = evo::evo_fwd_tri_kernel<D, HAS_PAIR>;
+    static AttrOnce attr;
+    if (!attr.ensure(dev, kernel, C::SMEM_BYTES)) return EVO_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return EVO_ERR_CUDA;
+    CUtensorMap tq, tk, tv, tp;
+    std::memset(&tp, 0, sizeof(tp));
+    if (!encode_qkv(&tq, Q, B * N, S, H, D) || !encode_qkv(&tk, K, B * N, S, H, D) ||
+        !encode_qkv(&tv, V, B * N, S, H, D))
+        return EVO_ERR_CUDA;
+    if (HAS_PAIR && !encode_pair(&tp, pair, B * H, S)) return EVO_ERR_CUDA;
+
+    evo::TriParams p;
+    p.mask = static_cast<const uint16_t*>(mask);
+    p.out = static_cast<uint16_t*>(O);
+    p.lse = LSE;
+    p.N = int(N);
+    p.S = int(S);
+    p.H = int(H);
+    p.num_kb = int((S + evo::kBN - 1) / evo::kBN);
+    p.num_qb = int((S + evo::kBM - 1) / evo::kBM);
+    p.num_n3 = int((N + 2) / 3);
+    p.num_tiles = int(int64_t(p.num_qb) * H * p.num_n3 * B);
+    p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
+    p.sqrt_d = float(std::sqrt(double(D)));
+    // the mask (or -inf for keys past S in a ragged last block) enters the score MMA
+    p.aug = (mask != nullptr || S % evo::kBN != 0) ? 1 : 0;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(p.num_tiles < sms ? p.num_tiles : sms), 1, 1);
+    cfg.blockDim = dim3(evo::kTriThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, tp, p) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+}
+
 // The SIMT kernel: T = float for fp32 inputs, uint16_t (bf16 bits) for the
 // bf16 shapes the tensor-core kernel does not take.
 template <typename T>
@@ -317,11 +362,15 @@ int launch_fwd(int dev, bool tensor_core, const void* Q, const void* K, const vo
 #define EVO_LAUNCH(DD)                                                                                \
     return has_pair ? launch_bf16<DD, true>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st) \
                     : launch_bf16<DD, false>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st)
+#define EVO_LAUNCH_TRI(DD)                                                                            \
+    return has_pair ? launch_tri<DD, true>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st) \
+                    : launch_tri<DD, false>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st)
     switch (D) {
-        case 16: EVO_LAUNCH(16);
-        case 32: EVO_LAUNCH(32);
+        case 16: EVO_LAUNCH_TRI(16);
+        case 32: EVO_LAUNCH_TRI(32);
         default: EVO_LAUNCH(64);
     }
+#undef EVO_LAUNCH_TRI
 #undef EVO_LAUNCH
 }
 

@@ -68,6 +68,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "common.cuh"
@@ -102,6 +103,9 @@ static_assert(128 * kHelperRegs + 256 * kSoftmaxRegs <= 384 * 168, "register spl
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 12.0f;  // log2 units: p <= 2^12 (fp16 P) between rescales
+// Masks more than this far below a row's running mask maximum (natural-log
+// units) are treated as -inf; see the mask-column writers.
+constexpr float kMaskFloor = 16384.0f;
 
 
 // UMMA shared-memory descriptor layout codes for swizzle spans of 32/64/128 B.
@@ -221,10 +225,10 @@ __device__ __forceinline__ uint32_t swz_chunk(int r, int c) {
 // the tile's chunk l + 32 g) of a V tile, bf16 -> fp16 in place (same
 // swizzled positions), by one warp; then the async-proxy fence that makes the
 // generic writes visible to the tensor cores.
-template <int FIRST, int COUNT>
+template <int FIRST, int COUNT, bool ROLLED = false>
 __device__ __forceinline__ void convert_v_chunks(uint32_t tile, int lane) {
     static_assert(FIRST % 4 == 0 && COUNT % 4 == 0, "whole groups of four");
-#pragma unroll
+#pragma unroll(ROLLED ? 1 : COUNT / 4)
     for (int g = FIRST; g < FIRST + COUNT; g += 4) {
         uint4 vv[4];
 #pragma unroll
@@ -459,7 +463,10 @@ evo_fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     for (int k = 0; k < 4; ++k) {
                         const int key = lane + 32 * k;
                         // (mask - c) * sqrt(D) as hi + mid + lo, three bf16 that sum to the fp32 value
-                        const float x = (v[k] - csub) * p.sqrt_d;
+                        // A key whose mask lies more than kMaskFloor below c weighs exactly
+                        // zero (e^-16384 underflows fp32 and fp64 alike): it enters as -inf, so
+                        // that no logit near -1e9 ever meets a running maximum near -1e9.
+                        const float x = (v[k] - csub < -kMaskFloor) ? -INFINITY : (v[k] - csub) * p.sqrt_d;
                         const uint32_t hi = ptx::f32_to_bf16_bits(x);
                         uint32_t mid = 0, lo = 0;
                         if (fabsf(x) < INFINITY) {
