@@ -85,18 +85,19 @@ struct TriCfg {
     static_assert(D == 16 || D == 32, "head dim");
     static constexpr int ROW = D * 2;                 // bytes per Q/K/V row = swizzle span
     static constexpr int TILE = kBM * ROW;            // one Q, K or V tile
+    static constexpr int Q_BUFS = 2;                  // per slice: this tile's Q and the next one's
     static constexpr int K_STAGES = 2;                // per slice
     static constexpr int V_STAGES = 2;                // per slice
     static constexpr int V_CHUNKS = TILE / 16 / 32;   // 16 B chunks per lane of a V tile
     static constexpr int AUG_ROW = 32;                // mask columns: 16 bf16 per row
     static constexpr int AUG_TILE = kBM * AUG_ROW;
-    static constexpr int M_STAGES = 2;                // mask-column tiles per slice
+    static constexpr int M_STAGES = 1;                // mask-column tiles per slice
     static constexpr int BIAS_BYTES = kBM * kBN * 2;  // two 128x64 boxes, 128 B swizzle
     static constexpr int B_STAGES = HAS_PAIR ? 2 : 0;
     static constexpr int B_RING = HAS_PAIR ? 2 : 1;   // ring arithmetic (no bias tiles without a pair bias)
     // shared-memory map (offsets from a 1024-aligned base; every tile 1024-aligned)
-    static constexpr int OFF_Q = 0;                                        // [3]
-    static constexpr int OFF_QAUG = OFF_Q + kTriSlices * TILE;
+    static constexpr int OFF_Q = 0;                                        // [3][Q_BUFS]
+    static constexpr int OFF_QAUG = OFF_Q + kTriSlices * Q_BUFS * TILE;
     static constexpr int OFF_K = OFF_QAUG + AUG_TILE;                      // [3][K_STAGES]
     static constexpr int OFF_V = OFF_K + kTriSlices * K_STAGES * TILE;     // [3][V_STAGES]
     static constexpr int OFF_KAUG = OFF_V + kTriSlices * V_STAGES * TILE;  // [3][M_STAGES]
@@ -104,8 +105,8 @@ struct TriCfg {
     static constexpr int OFF_MC = OFF_BIAS + B_STAGES * BIAS_BYTES;        // [3][M_STAGES] f32 rebase c
     static constexpr int OFF_BAR = OFF_MC + 64;
     // barrier indices (per slice w unless noted)
-    static constexpr int BAR_QF = 0;                                       // [3] Q tile landed
-    static constexpr int BAR_KF = BAR_QF + kTriSlices;                     // [3][K_STAGES] K landed
+    static constexpr int BAR_QF = 0;                                       // [3][Q_BUFS] Q tile landed
+    static constexpr int BAR_KF = BAR_QF + kTriSlices * Q_BUFS;            // [3][K_STAGES] K landed
     static constexpr int BAR_KE = BAR_KF + kTriSlices * K_STAGES;          // [3][K_STAGES] Q K^T done
     static constexpr int BAR_VF = BAR_KE + kTriSlices * K_STAGES;          // [3][V_STAGES] V landed (bf16)
     static constexpr int BAR_VE = BAR_VF + kTriSlices * V_STAGES;          // [3][V_STAGES] P.V done
@@ -113,9 +114,10 @@ struct TriCfg {
     static constexpr int BAR_BE = BAR_BF + 2;                              // [2] bias tile read by 12 softmax warps
     static constexpr int BAR_MF = BAR_BE + 2;                              // [3][M_STAGES] mask columns written
     static constexpr int BAR_ME = BAR_MF + kTriSlices * M_STAGES;          // [3][M_STAGES] read by MMA + softmax
-    static constexpr int BAR_SF = BAR_ME + kTriSlices * M_STAGES;          // [3] S ready
-    static constexpr int BAR_PF = BAR_SF + kTriSlices;                     // [3] P written
-    static constexpr int BAR_PE = BAR_PF + kTriSlices;                     // [3] last P.V of a tile done
+    static constexpr int BAR_SF = BAR_ME + kTriSlices * M_STAGES;          // [3][2] S of keys 0-63 / 64-127 ready
+    static constexpr int BAR_PF = BAR_SF + 2 * kTriSlices;                 // [3][2] P of keys 0-63 / 64-127 written
+    static constexpr int BAR_OA = BAR_PF + 2 * kTriSlices;                 // [3] P.V of keys 0-63 done
+    static constexpr int BAR_PE = BAR_OA + kTriSlices;                     // [3] last P.V of a tile done
     static constexpr int BAR_DRAIN = BAR_PE + kTriSlices;                  // [3] a helper's MMAs, on abort
     static constexpr int NUM_BARS = BAR_DRAIN + kTriSlices;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;    // tmem slot, abort flag
@@ -130,8 +132,9 @@ struct TriCfg {
     static constexpr uint32_t TMEM_COLS = 512;
     static_assert(TM_O0 + kTriSlices * D <= TMEM_COLS, "tensor memory");
     // instruction descriptors, fp32 accumulate, M = 128
+    // Q K^T of one half block: bf16 x bf16, both K-major, N = 64 keys
     static constexpr uint32_t IDESC_QK =
-        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(kBN) >> 3) << 17) | ((uint32_t(kBM) >> 4) << 24);
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(kBN / 2) >> 3) << 17) | ((uint32_t(kBM) >> 4) << 24);
     static constexpr uint32_t IDESC_PV =
         (1u << 4) | (0u << 7) | (0u << 10) | (1u << 16) | ((uint32_t(D) >> 3) << 17) | ((uint32_t(kBM) >> 4) << 24);
 };
@@ -185,7 +188,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     if (threadIdx.x == 0) {
         for (int w = 0; w < kTriSlices; ++w) {
-            ptx::mbar_init(bar(C::BAR_QF + w), 1);
+            for (int qb = 0; qb < C::Q_BUFS; ++qb) ptx::mbar_init(bar(C::BAR_QF + w * C::Q_BUFS + qb), 1);
             for (int st = 0; st < C::K_STAGES; ++st) {
                 ptx::mbar_init(bar(C::BAR_KF + w * C::K_STAGES + st), 1);
                 ptx::mbar_init(bar(C::BAR_KE + w * C::K_STAGES + st), 1);
@@ -198,8 +201,11 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ptx::mbar_init(bar(C::BAR_MF + w * C::M_STAGES + st), 1);
                 ptx::mbar_init(bar(C::BAR_ME + w * C::M_STAGES + st), 1 + 4);  // the MMA's commit + 4 softmax warps
             }
-            ptx::mbar_init(bar(C::BAR_SF + w), 1);
-            ptx::mbar_init(bar(C::BAR_PF + w), 4);
+            for (int hf = 0; hf < 2; ++hf) {
+                ptx::mbar_init(bar(C::BAR_SF + 2 * w + hf), 1);
+                ptx::mbar_init(bar(C::BAR_PF + 2 * w + hf), 4);
+            }
+            ptx::mbar_init(bar(C::BAR_OA + w), 1);
             ptx::mbar_init(bar(C::BAR_PE + w), 1);
             ptx::mbar_init(bar(C::BAR_DRAIN + w), 1);
         }
@@ -373,8 +379,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 q0 = t.qb * kBM;
                 bn = t.b * p.N + t.n0 + w;
             };
-            const uint32_t q_tile = sb + C::OFF_Q + uint32_t(w * C::TILE);
-            const uint64_t a_q = desc_k_major<C::ROW>(q_tile);
+            auto q_tile = [&](int qb) -> uint32_t { return sb + C::OFF_Q + uint32_t((w * C::Q_BUFS + qb) * C::TILE); };
             const uint64_t a_aug = desc_k_major<C::AUG_ROW>(sb + C::OFF_QAUG);
             const uint32_t d_s = tmem + C::TM_S0 + 128u * w;
             const uint32_t d_o = tmem + C::TM_O0 + uint32_t(D) * w;
@@ -392,35 +397,60 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const int st = n % C::V_STAGES;
                 ptx::tma_load_4d_elect(v_tile(st), &tm_v, bar(C::BAR_VF + w * C::V_STAGES + st), C::TILE, 0, h, j * kBN, bn);
             };
-            auto load_q = [&](int L) {
+            // Q of the slice's tile number tq (its buffer tq % 2)
+            auto load_q = [&](int L, int tq) {
                 int h, q0, bn;
                 coords(L, h, q0, bn);
-                ptx::tma_load_4d_elect(q_tile, &tm_q, bar(C::BAR_QF + w), C::TILE, 0, h, q0, bn);
+                const int qb = tq % C::Q_BUFS;
+                ptx::tma_load_4d_elect(q_tile(qb), &tm_q, bar(C::BAR_QF + w * C::Q_BUFS + qb), C::TILE, 0, h, q0, bn);
             };
             int n = 0, q_loads = 0, k_loads = 0, v_loads = 0;
+            int tcur = 0;  // the slice's tile number of stream position n
             bool issued_any = false;
-            // Q K^T of stream position n (block j of its tile), once K(n), the
-            // mask columns and (first block of a tile) Q are in place
-            auto issue_qk = [&](int nn, int j) -> bool {
+            // Q K^T of stream position n (block j of its tile) for keys 64 hf ..
+            // 64 hf + 63, into S columns 64 hf ..; the first half waits for K(n),
+            // the mask columns and (first block of a tile) Q
+            auto issue_qk = [&](int nn, int j, int hf, int tq) -> bool {
                 const int st = nn % C::K_STAGES;
-                if (j == 0 && !wait_warp(bar(C::BAR_QF + w), (q_loads - 1) & 1, abort_flag)) return false;
-                if (!wait_warp(bar(C::BAR_KF + w * C::K_STAGES + st), (nn / C::K_STAGES) & 1, abort_flag)) return false;
                 const int ms = w * C::M_STAGES + nn % C::M_STAGES;
-                if (aug && !wait_warp(bar(C::BAR_MF + ms), (nn / C::M_STAGES) & 1, abort_flag)) return false;
-                ptx::tc_fence_after();
-                const uint64_t bd = desc_k_major<C::ROW>(k_tile(st));
+                const int qb = tq % C::Q_BUFS;
+                const uint64_t a_q = desc_k_major<C::ROW>(q_tile(qb));
+                if (hf == 0) {
+                    if (j == 0 && !wait_warp(bar(C::BAR_QF + w * C::Q_BUFS + qb), (tq / C::Q_BUFS) & 1, abort_flag))
+                        return false;
+                    if (!wait_warp(bar(C::BAR_KF + w * C::K_STAGES + st), (nn / C::K_STAGES) & 1, abort_flag))
+                        return false;
+                    if (aug && !wait_warp(bar(C::BAR_MF + ms), (nn / C::M_STAGES) & 1, abort_flag)) return false;
+                    ptx::tc_fence_after();
+                }
+                const uint64_t bd = desc_k_major<C::ROW>(k_tile(st) + uint32_t(hf * 64 * C::ROW));
+                const uint32_t d = d_s + 64u * hf;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    ptx::mma_ss_elect(d_s, a_q + uint64_t(2 * kk), bd + uint64_t(2 * kk), C::IDESC_QK, kk > 0 ? 1u : 0u);
-                if (aug) {
-                    ptx::mma_ss_elect(d_s, a_aug, desc_k_major<C::AUG_ROW>(sb + C::OFF_KAUG + ms * C::AUG_TILE),
+                    ptx::mma_ss_elect(d, a_q + uint64_t(2 * kk), bd + uint64_t(2 * kk), C::IDESC_QK, kk > 0 ? 1u : 0u);
+                if (aug)
+                    ptx::mma_ss_elect(d, a_aug,
+                                      desc_k_major<C::AUG_ROW>(sb + C::OFF_KAUG + ms * C::AUG_TILE + hf * 64 * C::AUG_ROW),
                                       C::IDESC_QK, 1u);
-                    ptx::mma_commit_elect(bar(C::BAR_ME + ms));
+                if (hf == 1) {
+                    if (aug) ptx::mma_commit_elect(bar(C::BAR_ME + ms));
+                    ptx::mma_commit_elect(bar(C::BAR_KE + w * C::K_STAGES + st));
                 }
-                ptx::mma_commit_elect(bar(C::BAR_KE + w * C::K_STAGES + st));
-                ptx::mma_commit_elect(bar(C::BAR_SF + w));
+                ptx::mma_commit_elect(bar(C::BAR_SF + 2 * w + hf));
                 issued_any = true;
                 return true;
+            };
+            // P.V of keys 64 hf .. 64 hf + 63 of stream position n
+            auto issue_pv = [&](int nn, int j, int hf) {
+                const int st = nn % C::V_STAGES;
+                const uint64_t bd = desc_mn_major<C::ROW>(v_tile(st), uint32_t(C::TILE));
+#pragma unroll
+                for (int kk = 0; kk < kBN / 32; ++kk) {  // 16 keys per K step = 16 rows of V
+                    // keys 64 hf + 16 kk .. +15: P in columns 64 hf + 8 kk .. (fp16 pairs), V rows key0 ..
+                    const int key0 = 64 * hf + 16 * kk;
+                    ptx::mma_ts_elect(d_o, d_s + uint32_t(64 * hf + 8 * kk), bd + uint64_t((key0 * C::ROW) >> 4),
+                                      C::IDESC_PV, (j > 0 || hf > 0 || kk > 0) ? 1u : 0u);
+                }
             };
             int L = 0, j = 0;
             bool ok = first_pos(first_tile, L);
@@ -432,7 +462,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     ptx::prefetch_tmap(&tm_v);
                 }
                 __syncwarp();
-                load_q(L);
+                load_q(L, 0);
                 ++q_loads;
                 load_k(0, L, 0);
                 ++k_loads;
@@ -445,15 +475,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ++v_loads;
                 ok = wait_warp(bar(C::BAR_VF + w * C::V_STAGES), 0, abort_flag);
                 if (ok) convert_v_chunks<0, C::V_CHUNKS, true>(v_tile(0), lane);
-                ok = ok && issue_qk(0, 0);
-                if (ok && next_pos(L, 0, L1, j1) && j1 == 0) {
-                    // one key block per tile: position 1 needs the next Q as soon as Q K^T(0) is done
-                    ok = wait_warp(bar(C::BAR_KE + w * C::K_STAGES), 0, abort_flag);
-                    if (ok) {
-                        load_q(L1);
-                        ++q_loads;
-                    }
-                }
+                ok = ok && issue_qk(0, 0, 0, 0) && issue_qk(0, 0, 1, 0);
             }
             while (ok) {
                 int L1 = 0, j1 = 0, L2 = 0, j2 = 0;
@@ -467,36 +489,37 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     load_v(n + 1, L1, j1);
                     ++v_loads;
                 }
-                // P.V(n)
-                ok = wait_warp(bar(C::BAR_PF + w), n & 1, abort_flag);
+                const int tnext = (has1 && j1 == 0) ? tcur + 1 : tcur;  // tile number of position n+1
+                // keys 0-63 of block n: P.V, then Q K^T of keys 0-63 of block n+1
+                ok = wait_warp(bar(C::BAR_PF + 2 * w), n & 1, abort_flag);
                 if (!ok) break;
                 ptx::tc_fence_after();
-                {
-                    const int st = n % C::V_STAGES;
-                    const uint64_t bd = desc_mn_major<C::ROW>(v_tile(st), uint32_t(C::TILE));
-#pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)  // 16 keys per K step = 16 rows of V
-                        ptx::mma_ts_elect(d_o, d_s + 8u * kk, bd + uint64_t((16 * C::ROW * kk) >> 4), C::IDESC_PV,
-                                          (j > 0 || kk > 0) ? 1u : 0u);
-                    ptx::mma_commit_elect(bar(C::BAR_VE + w * C::V_STAGES + st));
-                    if (j == nkb - 1) ptx::mma_commit_elect(bar(C::BAR_PE + w));
+                issue_pv(n, j, 0);
+                ptx::mma_commit_elect(bar(C::BAR_OA + w));
+                if (j == 0) {
+                    // First block of a tile: every Q K^T of the previous tile is
+                    // complete (the softmax has seen S(n)), so its Q buffer takes
+                    // the next tile's Q, which then lands during this tile.
+                    int Ln;
+                    if (first_pos(L + G, Ln)) {
+                        load_q(Ln, tcur + 1);
+                        ++q_loads;
+                    }
                 }
-                if (!has1) break;
-                // Q K^T(n+1), then K(n+2) into the stage of K(n)
-                ok = issue_qk(n + 1, j1);
+                if (has1 && !issue_qk(n + 1, j1, 0, tnext)) { ok = false; break; }
+                // keys 64-127 of block n: P.V, then Q K^T of keys 64-127 of block n+1
+                ok = wait_warp(bar(C::BAR_PF + 2 * w + 1), n & 1, abort_flag);
                 if (!ok) break;
+                ptx::tc_fence_after();
+                issue_pv(n, j, 1);
+                ptx::mma_commit_elect(bar(C::BAR_VE + w * C::V_STAGES + n % C::V_STAGES));
+                if (j == nkb - 1) ptx::mma_commit_elect(bar(C::BAR_PE + w));
+                if (!has1) break;
+                if (!issue_qk(n + 1, j1, 1, tnext)) { ok = false; break; }
+                // K(n+2) into the stage of K(n) (Q K^T(n) is complete: the softmax saw S(n))
                 if (has2) {
                     load_k(n + 2, L2, j2);
                     ++k_loads;
-                    if (j2 == 0) {
-                        // Q of the next tile: the Q tile is free once Q K^T(n+1),
-                        // the last one of this tile, is done
-                        const int st = (n + 1) % C::K_STAGES;
-                        ok = wait_warp(bar(C::BAR_KE + w * C::K_STAGES + st), ((n + 1) / C::K_STAGES) & 1, abort_flag);
-                        if (!ok) break;
-                        load_q(L2);
-                        ++q_loads;
-                    }
                 }
                 // V(n+1) to fp16
                 {
@@ -507,6 +530,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 L = L1;
                 j = j1;
+                tcur = tnext;
                 ++n;
             }
             if (!ok && has_work) {
@@ -517,7 +541,8 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     wait_warp(bar(C::BAR_DRAIN + w), 0, nullptr);
                 }
                 if (lane == 0) {
-                    if (q_loads > 0) wait_bounded(bar(C::BAR_QF + w), (q_loads - 1) & 1, nullptr);
+                    for (int i2 = (q_loads > C::Q_BUFS ? q_loads - C::Q_BUFS : 0); i2 < q_loads; ++i2)
+                        wait_bounded(bar(C::BAR_QF + w * C::Q_BUFS + i2 % C::Q_BUFS), (i2 / C::Q_BUFS) & 1, nullptr);
                     for (int i2 = (k_loads > C::K_STAGES ? k_loads - C::K_STAGES : 0); i2 < k_loads; ++i2)
                         wait_bounded(bar(C::BAR_KF + w * C::K_STAGES + i2 % C::K_STAGES), (i2 / C::K_STAGES) & 1, nullptr);
                     for (int i2 = (v_loads > C::V_STAGES ? v_loads - C::V_STAGES : 0); i2 < v_loads; ++i2)
@@ -559,9 +584,20 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             float c_cur = 0.f;     // mask rebase that m and the stored P are relative to
             float2 suma = make_float2(0.f, 0.f), sumb = make_float2(0.f, 0.f);
             for (int j = 0; j < nkb && ok; ++j, ++blk) {
-                ok = wait_warp(bar(C::BAR_SF + w), blk & 1, abort_flag);
+                // S of keys 0-63 (keys 64-127 are waited for at step 2)
+                ok = wait_warp(bar(C::BAR_SF + 2 * w), blk & 1, abort_flag);
                 if (!ok) break;
                 ptx::tc_fence_after();
+                bool half_b_ready = false;  // S of keys 64-127 of this block waited for
+                // Waits for S of keys 64-127: after it, P.V of keys 64-127 of the
+                // previous block (issued just before that Q K^T) is complete.
+                auto wait_half_b = [&]() -> bool {
+                    if (half_b_ready) return true;
+                    if (!wait_warp(bar(C::BAR_SF + 2 * w + 1), blk & 1, abort_flag)) return false;
+                    ptx::tc_fence_after();
+                    half_b_ready = true;
+                    return true;
+                };
                 float s[32];  // one 32-key step of S(j), then t in place
                 if (aug) {
                     const int ms = w * C::M_STAGES + m_seen % C::M_STAGES;
@@ -601,8 +637,20 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // body, with its rare path, stays small enough for the
                 // instruction cache that the softmax warpgroups and the helpers
                 // share.
+                // P of step c goes to columns 16 c (keys 0-63) or 64 + 16 (c - 2)
+                // (keys 64-127): each over scores of its own half already read,
+                // so that Q K^T of keys 0-63 of the next block may overwrite
+                // columns 0-63 while the P of keys 64-127 waits for its P.V.
+                auto pcol = [](int c) -> uint32_t { return uint32_t(c < 2 ? 16 * c : 64 + 16 * (c - 2)); };
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
+                    if (c == 2) {
+                        // hand P of keys 0-63 to the tensor core, then wait for S of keys 64-127
+                        ptx::tmem_st_wait();
+                        ptx::tc_fence_before();
+                        ptx::mbar_arrive_elect(bar(C::BAR_PF + 2 * w));
+                        if (!(ok = wait_half_b())) break;
+                    }
                     tmem_ld_x32f(tS + 32u * c, s);
                     uint4 bw[4];
                     load_bias(c, bw);
@@ -673,11 +721,12 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         sumb = make_float2(sumb.x * alpha, sumb.y * alpha);
                         if (__any_sync(0xffffffffu, alpha != 1.f)) {
                             ptx::tmem_st_wait();
-                            // P of this block's earlier steps (fp16, 16 columns per step)
+                            // P of this block's earlier steps that the tensor core
+                            // has not taken yet (fp16, 16 columns per step)
 #pragma unroll 1
-                            for (int k = 0; k < c; ++k) {
+                            for (int k = (c < 2 ? 0 : 2); k < c; ++k) {
                                 uint32_t ok16[16];
-                                ptx::tmem_ld_x16(tS + 16u * k, ok16);
+                                ptx::tmem_ld_x16(tS + pcol(k), ok16);
                                 ptx::tmem_ld_wait_x16(ok16);
 #pragma unroll
                                 for (int e = 0; e < 16; ++e) {
@@ -685,10 +734,19 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                     const float2 f = __half22float2(h2);
                                     ok16[e] = ptx::pack_f16x2(f.x * alpha, f.y * alpha);
                                 }
-                                ptx::tmem_st_x16(tS + 16u * k, ok16);
+                                ptx::tmem_st_x16(tS + pcol(k), ok16);
                             }
-                            if (j > 0) {
-                                // O of the earlier blocks (P.V(j-1) is complete: S(j) landed after it)
+                            // O holds the earlier blocks and, from step 2 on, P.V of
+                            // keys 0-63 of this block; rescale it once the P.V
+                            // writing it are done: in steps 0-1 the last one is
+                            // keys 64-127 of the previous block, in steps 2-3 keys
+                            // 0-63 of this one.  (In block 0 before step 2, O holds
+                            // nothing yet: its first P.V overwrites it.)
+                            if (j > 0 || c >= 2) {
+                                bool ready = (c >= 2) ? wait_warp(bar(C::BAR_OA + w), blk & 1, abort_flag)
+                                                      : wait_half_b();
+                                if (!ready) { ok = false; break; }
+                                ptx::tc_fence_after();
                                 uint32_t o[D];
                                 if constexpr (D == 32) {
                                     ptx::tmem_ld_x32(tO, o);
@@ -723,12 +781,13 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                     suma = __fadd2_rn(suma, csa);
                     sumb = __fadd2_rn(sumb, csb);
-                    ptx::tmem_st_x8(tS + 16u * c, pk);
-                    ptx::tmem_st_x8(tS + 16u * c + 8u, pk + 8);
+                    ptx::tmem_st_x8(tS + pcol(c), pk);
+                    ptx::tmem_st_x8(tS + pcol(c) + 8u, pk + 8);
                 }
+                if (!ok) break;
                 ptx::tmem_st_wait();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive_elect(bar(C::BAR_PF + w));
+                ptx::mbar_arrive_elect(bar(C::BAR_PF + 2 * w + 1));
             }
             // -------------------------------------------------------- epilogue
             if (ok) ok = wait_warp(bar(C::BAR_PE + w), tiles & 1, abort_flag);
