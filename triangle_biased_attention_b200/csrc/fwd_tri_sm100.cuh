@@ -642,17 +642,20 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // so that Q K^T of keys 0-63 of the next block may overwrite
                 // columns 0-63 while the P of keys 64-127 waits for its P.V.
                 auto pcol = [](int c) -> uint32_t { return uint32_t(c < 2 ? 16 * c : 64 + 16 * (c - 2)); };
+                // S and the bias words of step c + 1 are requested as soon as step
+                // c no longer needs its registers (after its exps and its check),
+                // so their latency overlaps the stores of step c.
+                // Without a pair bias the S of step c + 1 is requested as soon as
+                // step c no longer needs its registers (after its exps and its
+                // check), so its latency overlaps the stores of step c.  With a
+                // pair bias, S and the bias words are requested at the top of
+                // each step (measured faster there).
+                constexpr bool kEarlyS = !HAS_PAIR;
+                if (kEarlyS) tmem_ld_x32f(tS, s);
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
-                    if (c == 2) {
-                        // hand P of keys 0-63 to the tensor core, then wait for S of keys 64-127
-                        ptx::tmem_st_wait();
-                        ptx::tc_fence_before();
-                        ptx::mbar_arrive_elect(bar(C::BAR_PF + 2 * w));
-                        if (!(ok = wait_half_b())) break;
-                    }
-                    tmem_ld_x32f(tS + 32u * c, s);
                     uint4 bw[4];
+                    if (!kEarlyS) tmem_ld_x32f(tS + 32u * c, s);
                     load_bias(c, bw);
                     tmem_wait_x32f(s);
                     // One basic block per step: t = S + pair * sqrt(D), the step
@@ -781,8 +784,20 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                     suma = __fadd2_rn(suma, csa);
                     sumb = __fadd2_rn(sumb, csb);
-                    ptx::tmem_st_x8(tS + pcol(c), pk);
-                    ptx::tmem_st_x8(tS + pcol(c) + 8u, pk + 8);
+                    if (c == 1) {
+                        // hand P of keys 0-63 to the tensor core, then wait for S of keys 64-127
+                        ptx::tmem_st_x8(tS + pcol(c), pk);
+                        ptx::tmem_st_x8(tS + pcol(c) + 8u, pk + 8);
+                        ptx::tmem_st_wait();
+                        ptx::tc_fence_before();
+                        ptx::mbar_arrive_elect(bar(C::BAR_PF + 2 * w));
+                        if (!(ok = wait_half_b())) break;
+                    }
+                    if (kEarlyS && c < 3) tmem_ld_x32f(tS + 32u * (c + 1), s);
+                    if (c != 1) {
+                        ptx::tmem_st_x8(tS + pcol(c), pk);
+                        ptx::tmem_st_x8(tS + pcol(c) + 8u, pk + 8);
+                    }
                 }
                 if (!ok) break;
                 ptx::tmem_st_wait();
