@@ -39,8 +39,8 @@ sys.path.insert(0, ROOT)
 from triangle_biased_attention_b200 import workloads as W  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-KERNEL_SOURCES = ["common.cuh", "ptx_sm100.cuh", "fwd_bf16_sm100.cuh", "evo_attn.cu"]
-KERNEL_NAME = "evo_fwd_bf16_kernel"
+KERNEL_SOURCES = ["common.cuh", "ptx_sm100.cuh", "tile_sm100.cuh", "fwd_tri_sm100.cuh", "evo_attn.cu"]
+KERNEL_NAME = "evo_fwd_tri_kernel"
 
 
 def parse():

@@ -82,9 +82,10 @@ def test_bf16_envelope(lib):
     # GPU that status marks an accepted shape.
     accepted = call()
     assert accepted == evo.EVO_ERR_INVALID_ARG
-    # head dims outside {16, 32, 64} up to 128, and pair biases whose rows are
-    # not whole 16-byte units, go to the SIMT kernel
-    for d in (1, 8, 24, 48, 128):
+    # head dims 16, 32, 64 and 128 go to the tensor-core kernel; other head
+    # dims up to 128, and pair biases whose rows are not whole 16-byte units,
+    # go to the SIMT kernel
+    for d in (1, 8, 24, 48, 64, 128):
         assert call(D=d) == accepted
     assert call(S=60, P=0x800000) == accepted
     for d in (129, 256):
@@ -95,13 +96,15 @@ def test_bf16_envelope(lib):
     assert call(D=48, Q=0x10001) == evo.EVO_ERR_MISALIGNED
     # the tensor-core shapes keep the 16-byte rule
     assert call(Q=0x10008) == evo.EVO_ERR_MISALIGNED
+    assert call(D=128, Q=0x10008) == evo.EVO_ERR_MISALIGNED
     assert call(O=0x100002) == evo.EVO_ERR_MISALIGNED
     assert call(P=0x800008) == evo.EVO_ERR_MISALIGNED
     assert call(M=0x900001) == evo.EVO_ERR_MISALIGNED
     assert call(L=0x200002) == evo.EVO_ERR_MISALIGNED
     far = dict(Q=1 << 50, K=2 << 50, V=3 << 50, O=4 << 50, L=5 << 50)
-    # CTA count = query blocks x heads x n pairs x batch beyond 2^31 - 1
-    assert call(B=1 << 15, N=1 << 10, S=1 << 10, H=1 << 4, D=16, **far) == evo.EVO_ERR_UNSUPPORTED_SHAPE
+    # tile count = query blocks x heads x n groups (3 slices at D = 16) x batch
+    # beyond 2^31 - 1
+    assert call(B=1 << 16, N=1 << 10, S=1 << 10, H=1 << 4, D=16, **far) == evo.EVO_ERR_UNSUPPORTED_SHAPE
 
 
 def test_fp32_envelope(lib):

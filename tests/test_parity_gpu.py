@@ -85,6 +85,11 @@ BF16_SHAPES = [
     (1, 2, 512, 2, 64, True, "bernoulli", 0, 0.01),
     (1, 3, 640, 2, 32, True, "head", 1, 0.0),      # leading blocks fully masked, then not
     (1, 2, 520, 1, 16, False, "head", 0, 0.0),     # same without pair bias, ragged S
+    (1, 2, 256, 2, 128, True, "bernoulli", 0, 0.01),  # D=128: two 128 B swizzle atoms per row
+    (1, 3, 136, 1, 128, False, "tail", 1, 0.0),    # D=128, ragged, no pair, a fully masked n
+    (2, 3, 384, 2, 64, True, "head", 1, 0.0),      # D=64 (two slices per tile), leading masked blocks
+    (1, 7, 128, 1, 64, True, "tail", 0, 0.0),      # D=64, odd N: a tile with one slice
+    (1, 4, 72, 2, 128, True, "none", 0, 0.0),      # D=128, S below one tile, S % 8 == 0 with pair bias
 ]
 
 
@@ -94,6 +99,7 @@ BF16_SHAPES = [
 SPIKE_SHAPES = [
     # B, N, S, H, D, mask, spike value, spike fraction, seed
     (1, 4, 512, 2, 32, "tail", 24.0, 0.002, 21),
+    (1, 2, 384, 1, 128, "bernoulli", 28.0, 0.002, 24),
     (1, 2, 640, 2, 64, "bernoulli", 30.0, 0.001, 22),
     (1, 3, 384, 1, 16, "tail", -40.0, 0.01, 23),
 ]
@@ -119,7 +125,7 @@ def test_bf16_random(shape):
 # bf16 inputs and output
 BF16_SIMT_SHAPES = [
     # B, N, S, H, D, pair, mask, fully_masked
-    (1, 3, 70, 2, 128, True, "tail", 1),   # D = 128, pair rows not 16-byte units
+    (1, 3, 70, 2, 128, True, "tail", 1),   # pair rows (S = 70) not 16-byte units
     (2, 2, 45, 3, 8, True, "tail", 0),     # small D, ragged S
     (1, 2, 130, 2, 48, False, "tail", 0),  # D not a multiple of 16
     (1, 4, 60, 2, 32, True, "tail", 0),    # D = 32 with S % 8 != 0 and a pair bias
@@ -142,7 +148,7 @@ def test_bf16_workload_full(name, seed):
 
 
 @pytest.mark.parametrize("seed", [0, 1])
-@pytest.mark.parametrize("name", ["msa_col_2048", "tri_1024", "tri_1024_d64"])
+@pytest.mark.parametrize("name", ["msa_col_2048", "tri_1024", "tri_1024_d64", "tri_512_d128"])
 def test_bf16_workload_sampled(name, seed):
     case = W.make_case(name, seed)
     slices = W.sample_slices(case, 64, seed, must_include_n=case.meta.get("fully_masked_n", []))

@@ -19,13 +19,11 @@
 
 #include "evo_attn.h"
 #include "common.cuh"
-#include "fwd_bf16_sm100.cuh"
 #include "fwd_tri_sm100.cuh"
 #include "fwd_f32.cuh"
 
 namespace {
 
-using evo::Bf16Cfg;
 
 constexpr int kMaxDevices = 64;
 
@@ -114,14 +112,15 @@ int select_device_of(const void* ptr, DeviceScope& scope) {
 }
 
 // Q/K/V/O as a 4-D tensor {D, H, S, B*N}; a box is one (b, n, h) slice's
-// 128 rows of D elements, swizzled over the D*2-byte row.
-bool encode_qkv(CUtensorMap* m, const void* base, int64_t BN, int64_t S, int64_t H, int64_t D) {
+// 128 rows of `box_w` elements (D, or 64 for D = 128, whose rows are loaded as
+// two boxes), swizzled over the box_w*2-byte row.
+bool encode_qkv(CUtensorMap* m, const void* base, int64_t BN, int64_t S, int64_t H, int64_t D, int64_t box_w) {
     const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(S), cuuint64_t(BN)};
     const cuuint64_t strides[3] = {cuuint64_t(D * 2), cuuint64_t(H * D * 2), cuuint64_t(S * H * D * 2)};
-    const cuuint32_t box[4] = {cuuint32_t(D), 1, cuuint32_t(evo::kBM), 1};
+    const cuuint32_t box[4] = {cuuint32_t(box_w), 1, cuuint32_t(evo::kBM), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
-                                          : (D == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    const CUtensorMapSwizzle sw = box_w == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                              : (box_w == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
     return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -139,48 +138,8 @@ bool encode_pair(CUtensorMap* m, const void* base, int64_t BH, int64_t S) {
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool HAS_PAIR>
-int launch_bf16(int dev, const void* Q, const void* K, const void* V, const void* mask, const void* pair, void* O,
-                float* LSE, int64_t B, int64_t N, int64_t S, int64_t H, cudaStream_t stream) {
-    using C = Bf16Cfg<D, HAS_PAIR>;
-    auto kernel = evo::evo_fwd_bf16_kernel<D, HAS_PAIR>;
-    static AttrOnce attr;
-    if (!attr.ensure(dev, kernel, C::SMEM_BYTES)) return EVO_ERR_CUDA;
-    CUtensorMap tq, tk, tv, tp;
-    std::memset(&tp, 0, sizeof(tp));
-    if (!encode_qkv(&tq, Q, B * N, S, H, D) || !encode_qkv(&tk, K, B * N, S, H, D) ||
-        !encode_qkv(&tv, V, B * N, S, H, D))
-        return EVO_ERR_CUDA;
-    if (HAS_PAIR && !encode_pair(&tp, pair, B * H, S)) return EVO_ERR_CUDA;
-
-    evo::Bf16Params p;
-    p.mask = static_cast<const uint16_t*>(mask);
-    p.out = static_cast<uint16_t*>(O);
-    p.lse = LSE;
-    p.N = int(N);
-    p.S = int(S);
-    p.H = int(H);
-    p.num_kb = int((S + evo::kBN - 1) / evo::kBN);
-    p.num_qb = int((S + evo::kBM - 1) / evo::kBM);
-    p.num_np = int((N + 1) / 2);
-    p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
-    p.sqrt_d = float(std::sqrt(double(D)));
-    // the mask (or -inf for keys past S in a ragged last block) enters the score MMA
-    p.aug = (mask != nullptr || S % evo::kBN != 0) ? 1 : 0;
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned(int64_t(p.num_qb) * H * p.num_np * B), 1, 1);
-    cfg.blockDim = dim3(evo::kThreads, 1, 1);
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
-    cfg.stream = stream;
-    cfg.attrs = nullptr;
-    cfg.numAttrs = 0;
-    return cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, tp, p) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
-}
-
-// The three-slice persistent kernel (head dims 16 and 32): one CTA per SM,
-// each walking the tiles (query block, head, n triple, batch) with a stride
-// of the grid size.
+// The tcgen05 kernel: one CTA per SM, each walking the tiles (query block,
+// head, group of n slices, batch) with a stride of the grid size.
 template <int D, bool HAS_PAIR>
 int launch_tri(int dev, const void* Q, const void* K, const void* V, const void* mask, const void* pair, void* O,
                float* LSE, int64_t B, int64_t N, int64_t S, int64_t H, cudaStream_t stream) {
@@ -193,8 +152,8 @@ int launch_tri(int dev, const void* Q, const void* K, const void* V, const void*
         return EVO_ERR_CUDA;
     CUtensorMap tq, tk, tv, tp;
     std::memset(&tp, 0, sizeof(tp));
-    if (!encode_qkv(&tq, Q, B * N, S, H, D) || !encode_qkv(&tk, K, B * N, S, H, D) ||
-        !encode_qkv(&tv, V, B * N, S, H, D))
+    if (!encode_qkv(&tq, Q, B * N, S, H, D, C::SUBW) || !encode_qkv(&tk, K, B * N, S, H, D, C::SUBW) ||
+        !encode_qkv(&tv, V, B * N, S, H, D, C::SUBW))
         return EVO_ERR_CUDA;
     if (HAS_PAIR && !encode_pair(&tp, pair, B * H, S)) return EVO_ERR_CUDA;
 
@@ -207,8 +166,8 @@ int launch_tri(int dev, const void* Q, const void* K, const void* V, const void*
     p.H = int(H);
     p.num_kb = int((S + evo::kBN - 1) / evo::kBN);
     p.num_qb = int((S + evo::kBM - 1) / evo::kBM);
-    p.num_n3 = int((N + 2) / 3);
-    p.num_tiles = int(int64_t(p.num_qb) * H * p.num_n3 * B);
+    p.num_ng = int((N + C::NS - 1) / C::NS);
+    p.num_tiles = int(int64_t(p.num_qb) * H * p.num_ng * B);
     p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
     p.sqrt_d = float(std::sqrt(double(D)));
     // the mask (or -inf for keys past S in a ragged last block) enters the score MMA
@@ -216,7 +175,7 @@ int launch_tri(int dev, const void* Q, const void* K, const void* V, const void*
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(unsigned(p.num_tiles < sms ? p.num_tiles : sms), 1, 1);
-    cfg.blockDim = dim3(evo::kTriThreads, 1, 1);
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
     return cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, tp, p) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
@@ -321,15 +280,15 @@ int check_fwd(const void* Q, const void* K, const void* V, const void* mask_bias
     // bf16 runs on the tensor-core kernel for D in {16, 32, 64} when the pair
     // bias rows are whole 16-byte units (S a multiple of 8); every other bf16
     // shape with D <= 128 runs on the SIMT kernel
-    *tensor_core =
-        dtype == EVO_DTYPE_BF16 && (D == 16 || D == 32 || D == 64) && !(pair_bias && (S % 8) != 0);
+    *tensor_core = dtype == EVO_DTYPE_BF16 && (D == 16 || D == 32 || D == 64 || D == 128) &&
+                   !(pair_bias && (S % 8) != 0);
     if (*tensor_core) {
         // TMA coordinates are 32-bit; the CTA count (query blocks x heads x
         // n pairs x batch) must fit the grid's x dimension
         int64_t ctas;
         if (bn > int_max || bh > int_max || S > int_max || N > int_max || H > int_max ||
-            !mul_ok((S + evo::kBM - 1) / evo::kBM, bh, &ctas) || !mul_ok(ctas, (N + 1) / 2, &ctas) ||
-            ctas > int_max)
+            !mul_ok((S + evo::kBM - 1) / evo::kBM, bh, &ctas) ||
+            !mul_ok(ctas, (N + evo::tri_slices(int(D)) - 1) / evo::tri_slices(int(D)), &ctas) || ctas > int_max)
             return EVO_ERR_UNSUPPORTED_SHAPE;
         if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) ||
             (pair_bias && !aligned(pair_bias, 16)) || (mask_bias && !aligned(mask_bias, 2)))
@@ -359,19 +318,16 @@ int launch_fwd(int dev, bool tensor_core, const void* Q, const void* K, const vo
 
     if (encode_fn() == nullptr) return EVO_ERR_CUDA;
     const bool has_pair = pair_bias != nullptr;
-#define EVO_LAUNCH(DD)                                                                                \
-    return has_pair ? launch_bf16<DD, true>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st) \
-                    : launch_bf16<DD, false>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st)
 #define EVO_LAUNCH_TRI(DD)                                                                            \
     return has_pair ? launch_tri<DD, true>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st) \
                     : launch_tri<DD, false>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st)
     switch (D) {
         case 16: EVO_LAUNCH_TRI(16);
         case 32: EVO_LAUNCH_TRI(32);
-        default: EVO_LAUNCH(64);
+        case 64: EVO_LAUNCH_TRI(64);
+        default: EVO_LAUNCH_TRI(128);
     }
 #undef EVO_LAUNCH_TRI
-#undef EVO_LAUNCH
 }
 
 // Every buffer of a call must live on Q's device; makes it current.

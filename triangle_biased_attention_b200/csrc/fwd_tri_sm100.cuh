@@ -53,7 +53,7 @@
 
 #include "common.cuh"
 #include "ptx_sm100.cuh"
-#include "fwd_bf16_sm100.cuh"  // descriptors, swizzle helpers, V conversion
+#include "tile_sm100.cuh"  // descriptors, swizzle helpers, V conversion
 
 namespace evo {
 
@@ -64,30 +64,45 @@ struct TriParams {
     int N, S, H;
     int num_kb;            // key blocks of 128
     int num_qb;            // query blocks of 128
-    int num_n3;            // n triples per batch entry, ceil(N / 3)
-    int num_tiles;         // B * num_n3 * H * num_qb
+    int num_ng;            // n groups per batch entry, ceil(N / slices per tile)
+    int num_tiles;         // B * num_ng * H * num_qb
     int aug;               // mask columns in the score MMA (a mask, or a ragged last key block)
     float scale_log2;      // log2(e) / sqrt(D)
     float sqrt_d;          // sqrt(D)
 };
 
-constexpr int kTriSlices = 3;
 // The running maximum moves when a step exceeds it by more than this (log2
 // units): p <= 2^15 keeps P inside fp16 (largest finite 65504).
 constexpr float kTriRescaleThreshold = 15.0f;
-constexpr int kTriThreads = 512;      // helper warpgroup + three softmax warpgroups
-constexpr int kTriHelperRegs = 80;
-constexpr int kTriSoftmaxRegs = 144;
-static_assert(128 * kTriHelperRegs + 3 * 128 * kTriSoftmaxRegs <= kTriThreads * 128, "register split");
+
+// Slices per tile: as many as tensor memory holds, each a 128-column score
+// buffer plus a D-column O accumulator.
+__host__ __device__ constexpr int tri_slices(int D) { return D <= 32 ? 3 : (D == 64 ? 2 : 1); }
 
 template <int D, bool HAS_PAIR>
 struct TriCfg {
-    static_assert(D == 16 || D == 32, "head dim");
-    static constexpr int ROW = D * 2;                 // bytes per Q/K/V row = swizzle span
-    static constexpr int TILE = kBM * ROW;            // one Q, K or V tile
-    static constexpr int Q_BUFS = 2;                  // per slice: this tile's Q and the next one's
-    static constexpr int K_STAGES = 2;                // per slice
-    static constexpr int V_STAGES = 2;                // per slice
+    static_assert(D == 16 || D == 32 || D == 64 || D == 128, "head dim");
+    static constexpr int NS = tri_slices(D);          // slices per tile
+    static constexpr int THREADS = 128 * (1 + NS);    // helper warpgroup + one softmax warpgroup per slice
+    // register split (setmaxnreg) where the launch leaves less than the
+    // softmax needs: the helper warpgroup hands registers to the softmax
+    static constexpr bool SPLIT_REGS = NS >= 2;
+    static constexpr int HELPER_REGS = NS == 3 ? 80 : 96;
+    static constexpr int SOFTMAX_REGS = NS == 3 ? 144 : 200;
+    static_assert(!SPLIT_REGS || 128 * HELPER_REGS + NS * 128 * SOFTMAX_REGS <= THREADS * (65536 / THREADS / 8 * 8),
+                  "register split");
+    // a Q/K/V row is D bf16; rows wider than 128 B are split into sub-tiles of
+    // 64 elements (one 128 B swizzle atom each)
+    static constexpr int SUBW = D <= 64 ? D : 64;     // elements per sub-tile row
+    static constexpr int NSUB = D / SUBW;             // sub-tiles per tile
+    static constexpr int ROW = SUBW * 2;              // bytes per sub-tile row = swizzle span
+    static constexpr int SUBTILE = kBM * ROW;
+    static constexpr int TILE = NSUB * SUBTILE;       // one Q, K or V tile
+    static constexpr int KPA = SUBW / 16;             // 16-element MMA K steps per swizzle atom
+    // stages per slice, as many as shared memory holds
+    static constexpr int Q_BUFS = D <= 32 ? 2 : 1;    // 2: this tile's Q and the next one's
+    static constexpr int K_STAGES = 2;
+    static constexpr int V_STAGES = D <= 32 ? 2 : 1;
     static constexpr int V_CHUNKS = TILE / 16 / 32;   // 16 B chunks per lane of a V tile
     static constexpr int AUG_ROW = 32;                // mask columns: 16 bf16 per row
     static constexpr int AUG_TILE = kBM * AUG_ROW;
@@ -96,30 +111,30 @@ struct TriCfg {
     static constexpr int B_STAGES = HAS_PAIR ? 2 : 0;
     static constexpr int B_RING = HAS_PAIR ? 2 : 1;   // ring arithmetic (no bias tiles without a pair bias)
     // shared-memory map (offsets from a 1024-aligned base; every tile 1024-aligned)
-    static constexpr int OFF_Q = 0;                                        // [3][Q_BUFS]
-    static constexpr int OFF_QAUG = OFF_Q + kTriSlices * Q_BUFS * TILE;
-    static constexpr int OFF_K = OFF_QAUG + AUG_TILE;                      // [3][K_STAGES]
-    static constexpr int OFF_V = OFF_K + kTriSlices * K_STAGES * TILE;     // [3][V_STAGES]
-    static constexpr int OFF_KAUG = OFF_V + kTriSlices * V_STAGES * TILE;  // [3][M_STAGES]
-    static constexpr int OFF_BIAS = OFF_KAUG + kTriSlices * M_STAGES * AUG_TILE;
-    static constexpr int OFF_MC = OFF_BIAS + B_STAGES * BIAS_BYTES;        // [3][M_STAGES] f32 rebase c
+    static constexpr int OFF_Q = 0;                                        // [NS][Q_BUFS]
+    static constexpr int OFF_QAUG = OFF_Q + NS * Q_BUFS * TILE;
+    static constexpr int OFF_K = OFF_QAUG + AUG_TILE;                      // [NS][K_STAGES]
+    static constexpr int OFF_V = OFF_K + NS * K_STAGES * TILE;     // [NS][V_STAGES]
+    static constexpr int OFF_KAUG = OFF_V + NS * V_STAGES * TILE;  // [NS][M_STAGES]
+    static constexpr int OFF_BIAS = OFF_KAUG + NS * M_STAGES * AUG_TILE;
+    static constexpr int OFF_MC = OFF_BIAS + B_STAGES * BIAS_BYTES;        // [NS][M_STAGES] f32 rebase c
     static constexpr int OFF_BAR = OFF_MC + 64;
     // barrier indices (per slice w unless noted)
-    static constexpr int BAR_QF = 0;                                       // [3][Q_BUFS] Q tile landed
-    static constexpr int BAR_KF = BAR_QF + kTriSlices * Q_BUFS;            // [3][K_STAGES] K landed
-    static constexpr int BAR_KE = BAR_KF + kTriSlices * K_STAGES;          // [3][K_STAGES] Q K^T done
-    static constexpr int BAR_VF = BAR_KE + kTriSlices * K_STAGES;          // [3][V_STAGES] V landed (bf16)
-    static constexpr int BAR_VE = BAR_VF + kTriSlices * V_STAGES;          // [3][V_STAGES] P.V done
-    static constexpr int BAR_BF = BAR_VE + kTriSlices * V_STAGES;          // [2] bias tile landed (shared)
+    static constexpr int BAR_QF = 0;                                       // [NS][Q_BUFS] Q tile landed
+    static constexpr int BAR_KF = BAR_QF + NS * Q_BUFS;            // [NS][K_STAGES] K landed
+    static constexpr int BAR_KE = BAR_KF + NS * K_STAGES;          // [NS][K_STAGES] Q K^T done
+    static constexpr int BAR_VF = BAR_KE + NS * K_STAGES;          // [NS][V_STAGES] V landed (bf16)
+    static constexpr int BAR_VE = BAR_VF + NS * V_STAGES;          // [NS][V_STAGES] P.V done
+    static constexpr int BAR_BF = BAR_VE + NS * V_STAGES;          // [2] bias tile landed (shared)
     static constexpr int BAR_BE = BAR_BF + 2;                              // [2] bias tile read by 12 softmax warps
-    static constexpr int BAR_MF = BAR_BE + 2;                              // [3][M_STAGES] mask columns written
-    static constexpr int BAR_ME = BAR_MF + kTriSlices * M_STAGES;          // [3][M_STAGES] read by MMA + softmax
-    static constexpr int BAR_SF = BAR_ME + kTriSlices * M_STAGES;          // [3][2] S of keys 0-63 / 64-127 ready
-    static constexpr int BAR_PF = BAR_SF + 2 * kTriSlices;                 // [3][2] P of keys 0-63 / 64-127 written
-    static constexpr int BAR_OA = BAR_PF + 2 * kTriSlices;                 // [3] P.V of keys 0-63 done
-    static constexpr int BAR_PE = BAR_OA + kTriSlices;                     // [3] last P.V of a tile done
-    static constexpr int BAR_DRAIN = BAR_PE + kTriSlices;                  // [3] a helper's MMAs, on abort
-    static constexpr int NUM_BARS = BAR_DRAIN + kTriSlices;
+    static constexpr int BAR_MF = BAR_BE + 2;                              // [NS][M_STAGES] mask columns written
+    static constexpr int BAR_ME = BAR_MF + NS * M_STAGES;          // [NS][M_STAGES] read by MMA + softmax
+    static constexpr int BAR_SF = BAR_ME + NS * M_STAGES;          // [NS][2] S of keys 0-63 / 64-127 ready
+    static constexpr int BAR_PF = BAR_SF + 2 * NS;                 // [NS][2] P of keys 0-63 / 64-127 written
+    static constexpr int BAR_OA = BAR_PF + 2 * NS;                 // [NS] P.V of keys 0-63 done
+    static constexpr int BAR_PE = BAR_OA + NS;                     // [NS] last P.V of a tile done
+    static constexpr int BAR_DRAIN = BAR_PE + NS;                  // [NS] a helper's MMAs, on abort
+    static constexpr int NUM_BARS = BAR_DRAIN + NS;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;    // tmem slot, abort flag
     static constexpr int USED = OFF_MISC + 16;
     // + alignment slack; at least 116 KB so that two CTAs never share an SM
@@ -128,9 +143,9 @@ struct TriCfg {
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
     // tensor-memory columns
     static constexpr uint32_t TM_S0 = 0;    // + 128 * w: S, with P over its first 64 columns
-    static constexpr uint32_t TM_O0 = 384;  // + D * w
-    static constexpr uint32_t TMEM_COLS = 512;
-    static_assert(TM_O0 + kTriSlices * D <= TMEM_COLS, "tensor memory");
+    static constexpr uint32_t TM_O0 = 128u * NS;  // + D * w
+    static constexpr uint32_t TMEM_COLS = (TM_O0 + NS * D) <= 256 ? 256u : 512u;
+    static_assert(TM_O0 + NS * D <= TMEM_COLS, "tensor memory");
     // instruction descriptors, fp32 accumulate, M = 128
     // Q K^T of one half block: bf16 x bf16, both K-major, N = 64 keys
     static constexpr uint32_t IDESC_QK =
@@ -144,16 +159,16 @@ struct TriTile {
     int qb, h, n0, b, nv;
 };
 
-__device__ __forceinline__ TriTile tri_tile(const TriParams& p, int L) {
+__device__ __forceinline__ TriTile tri_tile(const TriParams& p, int L, int ns) {
     TriTile t;
     t.qb = L % p.num_qb;
     int rest = L / p.num_qb;
     t.h = rest % p.H;
     rest /= p.H;
-    const int n3 = rest % p.num_n3;
-    t.b = rest / p.num_n3;
-    t.n0 = 3 * n3;
-    t.nv = (p.N - t.n0) < 3 ? (p.N - t.n0) : 3;
+    const int ng = rest % p.num_ng;
+    t.b = rest / p.num_ng;
+    t.n0 = ns * ng;
+    t.nv = (p.N - t.n0) < ns ? (p.N - t.n0) : ns;
     return t;
 }
 
@@ -163,7 +178,7 @@ __device__ __forceinline__ void tmem_ld_x32f(uint32_t taddr, float* f) {
 __device__ __forceinline__ void tmem_wait_x32f(float* f) { ptx::tmem_ld_wait_x32(reinterpret_cast<uint32_t*>(f)); }
 
 template <int D, bool HAS_PAIR>
-__global__ void __launch_bounds__(kTriThreads, 1)
+__global__ void __launch_bounds__(TriCfg<D, HAS_PAIR>::THREADS, 1)
 evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_pair,
                    const TriParams p) {
@@ -187,7 +202,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     float* mc_s = reinterpret_cast<float*>(smem + C::OFF_MC);  // [w * M_STAGES + stage]
 
     if (threadIdx.x == 0) {
-        for (int w = 0; w < kTriSlices; ++w) {
+        for (int w = 0; w < C::NS; ++w) {
             for (int qb = 0; qb < C::Q_BUFS; ++qb) ptx::mbar_init(bar(C::BAR_QF + w * C::Q_BUFS + qb), 1);
             for (int st = 0; st < C::K_STAGES; ++st) {
                 ptx::mbar_init(bar(C::BAR_KF + w * C::K_STAGES + st), 1);
@@ -211,7 +226,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         for (int st = 0; st < 2; ++st) {
             ptx::mbar_init(bar(C::BAR_BF + st), 1);
-            ptx::mbar_init(bar(C::BAR_BE + st), 4 * kTriSlices);
+            ptx::mbar_init(bar(C::BAR_BE + st), 4 * C::NS);
         }
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -219,7 +234,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     if (warp == 0) {
         // The A tile of the mask step: columns 0-2 = 1.0 (bf16), rest 0.  The
         // mask-column B tiles start zeroed; only columns 0-2 are rewritten.
-        for (int c = lane; c < (C::AUG_TILE * (1 + kTriSlices * C::M_STAGES)) / 16; c += 32) {
+        for (int c = lane; c < (C::AUG_TILE * (1 + C::NS * C::M_STAGES)) / 16; c += 32) {
             const uint32_t addr = (c < C::AUG_TILE / 16) ? sb + C::OFF_QAUG + uint32_t(c) * 16u
                                                          : sb + C::OFF_KAUG + uint32_t(c - C::AUG_TILE / 16) * 16u;
             ptx::st_shared_v4(addr, make_uint4(0u, 0u, 0u, 0u));
@@ -237,8 +252,10 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    if (warp < 4) ptx::setmaxnreg_dec<kTriHelperRegs>();
-    else ptx::setmaxnreg_inc<kTriSoftmaxRegs>();
+    if constexpr (C::SPLIT_REGS) {
+        if (warp < 4) ptx::setmaxnreg_dec<C::HELPER_REGS>();
+        else ptx::setmaxnreg_inc<C::SOFTMAX_REGS>();
+    }
 
     if (warp < 4) {
         if (warp == 0) {
@@ -253,13 +270,15 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if (lane == 0) {
                 ptx::prefetch_tmap(&tm_pair);
             }
-            int b_issued = 0, m_done[kTriSlices] = {0, 0, 0};
-            float c_run[kTriSlices] = {-INFINITY, -INFINITY, -INFINITY};
-            uint32_t raw[kTriSlices][4];
-            auto fetch = [&](int L, int j) {
-                const TriTile t = tri_tile(p, L);
+            int b_issued = 0, m_done[C::NS] = {};
+            float c_run[C::NS];
 #pragma unroll
-                for (int w = 0; w < kTriSlices; ++w) {
+            for (int w = 0; w < C::NS; ++w) c_run[w] = -INFINITY;
+            uint32_t raw[C::NS][4];
+            auto fetch = [&](int L, int j) {
+                const TriTile t = tri_tile(p, L, C::NS);
+#pragma unroll
+                for (int w = 0; w < C::NS; ++w) {
                     const uint16_t* mrow = (p.mask != nullptr && w < t.nv)
                                                ? p.mask + (size_t(t.b) * p.N + t.n0 + w) * size_t(p.S)
                                                : nullptr;
@@ -273,7 +292,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             bool ok = true;
             if (aug) fetch(first_tile, 0);
             for (int it = 0, L = first_tile; L < p.num_tiles && ok; ++it, L += G) {
-                const TriTile t = tri_tile(p, L);
+                const TriTile t = tri_tile(p, L, C::NS);
                 for (int j = 0; j < nkb && ok; ++j) {
                     if (HAS_PAIR) {
                         const int st = b_issued % C::B_RING;
@@ -290,15 +309,15 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         ++b_issued;
                     }
                     if (!aug) continue;
-                    uint32_t cur[kTriSlices][4];
+                    uint32_t cur[C::NS][4];
 #pragma unroll
-                    for (int w = 0; w < kTriSlices; ++w)
+                    for (int w = 0; w < C::NS; ++w)
 #pragma unroll
                         for (int k = 0; k < 4; ++k) cur[w][k] = raw[w][k];
                     if (j + 1 < nkb) fetch(L, j + 1);
                     else if (L + G < p.num_tiles) fetch(L + G, 0);
 #pragma unroll
-                    for (int w = 0; w < kTriSlices; ++w) {
+                    for (int w = 0; w < C::NS; ++w) {
                         if (!ok || w >= t.nv) break;
                         if (j == 0) c_run[w] = -INFINITY;
                         float v[4];
@@ -348,7 +367,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     wait_bounded(bar(C::BAR_BF + i2 % C::B_RING), (i2 / C::B_RING) & 1, nullptr);
             }
             __syncwarp();
-        } else {
+        } else if (warp - 1 < C::NS) {
             // ------------------------------------------- helper of slice w
             // Warp 1 + w drives slice n0 + w through every tile that has it:
             // its Q, K and V loads, the conversion of its V tiles to fp16, and
@@ -365,7 +384,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // the slice's stream: position = (tile index L, key block j)
             auto first_pos = [&](int L, int& outL) -> bool {
                 for (; L < p.num_tiles; L += G)
-                    if (w < tri_tile(p, L).nv) { outL = L; return true; }
+                    if (w < tri_tile(p, L, C::NS).nv) { outL = L; return true; }
                 return false;
             };
             auto next_pos = [&](int L, int j, int& nL, int& nj) -> bool {
@@ -374,7 +393,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 return first_pos(L + G, nL);
             };
             auto coords = [&](int L, int& h, int& q0, int& bn) {
-                const TriTile t = tri_tile(p, L);
+                const TriTile t = tri_tile(p, L, C::NS);
                 h = t.h;
                 q0 = t.qb * kBM;
                 bn = t.b * p.N + t.n0 + w;
@@ -385,24 +404,31 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const uint32_t d_o = tmem + C::TM_O0 + uint32_t(D) * w;
             auto k_tile = [&](int st) -> uint32_t { return sb + C::OFF_K + uint32_t((w * C::K_STAGES + st) * C::TILE); };
             auto v_tile = [&](int st) -> uint32_t { return sb + C::OFF_V + uint32_t((w * C::V_STAGES + st) * C::TILE); };
+            // one tile = NSUB boxes of SUBW elements per row, one barrier
+            auto load_tile = [&](uint32_t dst, const CUtensorMap* m, uint32_t bar_addr, int h, int row0, int bn) {
+                ptx::tma_load_4d_elect(dst, m, bar_addr, uint32_t(C::TILE), 0, h, row0, bn);
+#pragma unroll
+                for (int sub = 1; sub < C::NSUB; ++sub)
+                    ptx::tma_load_4d_more_elect(dst + uint32_t(sub * C::SUBTILE), m, bar_addr, sub * C::SUBW, h, row0, bn);
+            };
             auto load_k = [&](int n, int L, int j) {
                 int h, q0, bn;
                 coords(L, h, q0, bn);
                 const int st = n % C::K_STAGES;
-                ptx::tma_load_4d_elect(k_tile(st), &tm_k, bar(C::BAR_KF + w * C::K_STAGES + st), C::TILE, 0, h, j * kBN, bn);
+                load_tile(k_tile(st), &tm_k, bar(C::BAR_KF + w * C::K_STAGES + st), h, j * kBN, bn);
             };
             auto load_v = [&](int n, int L, int j) {
                 int h, q0, bn;
                 coords(L, h, q0, bn);
                 const int st = n % C::V_STAGES;
-                ptx::tma_load_4d_elect(v_tile(st), &tm_v, bar(C::BAR_VF + w * C::V_STAGES + st), C::TILE, 0, h, j * kBN, bn);
+                load_tile(v_tile(st), &tm_v, bar(C::BAR_VF + w * C::V_STAGES + st), h, j * kBN, bn);
             };
-            // Q of the slice's tile number tq (its buffer tq % 2)
+            // Q of the slice's tile number tq (its buffer tq % Q_BUFS)
             auto load_q = [&](int L, int tq) {
                 int h, q0, bn;
                 coords(L, h, q0, bn);
                 const int qb = tq % C::Q_BUFS;
-                ptx::tma_load_4d_elect(q_tile(qb), &tm_q, bar(C::BAR_QF + w * C::Q_BUFS + qb), C::TILE, 0, h, q0, bn);
+                load_tile(q_tile(qb), &tm_q, bar(C::BAR_QF + w * C::Q_BUFS + qb), h, q0, bn);
             };
             int n = 0, q_loads = 0, k_loads = 0, v_loads = 0;
             int tcur = 0;  // the slice's tile number of stream position n
@@ -426,8 +452,11 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const uint64_t bd = desc_k_major<C::ROW>(k_tile(st) + uint32_t(hf * 64 * C::ROW));
                 const uint32_t d = d_s + 64u * hf;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    ptx::mma_ss_elect(d, a_q + uint64_t(2 * kk), bd + uint64_t(2 * kk), C::IDESC_QK, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    // K step kk: 32 B into its sub-tile's swizzled rows (descriptor units of 16 B)
+                    const uint64_t off = uint64_t((kk / C::KPA) * (C::SUBTILE >> 4) + 2 * (kk % C::KPA));
+                    ptx::mma_ss_elect(d, a_q + off, bd + off, C::IDESC_QK, kk > 0 ? 1u : 0u);
+                }
                 if (aug)
                     ptx::mma_ss_elect(d, a_aug,
                                       desc_k_major<C::AUG_ROW>(sb + C::OFF_KAUG + ms * C::AUG_TILE + hf * 64 * C::AUG_ROW),
@@ -443,7 +472,8 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // P.V of keys 64 hf .. 64 hf + 63 of stream position n
             auto issue_pv = [&](int nn, int j, int hf) {
                 const int st = nn % C::V_STAGES;
-                const uint64_t bd = desc_mn_major<C::ROW>(v_tile(st), uint32_t(C::TILE));
+                // V as the MN-major B operand: N = D in NSUB atoms SUBTILE bytes apart
+                const uint64_t bd = desc_mn_major<C::ROW>(v_tile(st), uint32_t(C::SUBTILE));
 #pragma unroll
                 for (int kk = 0; kk < kBN / 32; ++kk) {  // 16 keys per K step = 16 rows of V
                     // keys 64 hf + 16 kk .. +15: P in columns 64 hf + 8 kk .. (fp16 pairs), V rows key0 ..
@@ -476,13 +506,23 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ok = wait_warp(bar(C::BAR_VF + w * C::V_STAGES), 0, abort_flag);
                 if (ok) convert_v_chunks<0, C::V_CHUNKS, true>(v_tile(0), lane);
                 ok = ok && issue_qk(0, 0, 0, 0) && issue_qk(0, 0, 1, 0);
+                if (ok && C::Q_BUFS == 1 && next_pos(L, 0, L1, j1) && j1 == 0) {
+                    // one key block per tile and one Q buffer: position 1 needs the
+                    // next Q as soon as Q K^T(0) is done
+                    ok = wait_warp(bar(C::BAR_KE + w * C::K_STAGES), 0, abort_flag);
+                    if (ok) {
+                        load_q(L1, 1);
+                        ++q_loads;
+                    }
+                }
             }
             while (ok) {
                 int L1 = 0, j1 = 0, L2 = 0, j2 = 0;
                 const bool has1 = next_pos(L, j, L1, j1);
                 const bool has2 = has1 && next_pos(L1, j1, L2, j2);
-                // V(n+1) into the stage of V(n-1), once P.V(n-1) is done
-                if (has1) {
+                // V(n+1) into the stage of V(n-1), once P.V(n-1) is done (with one
+                // stage, after P.V(n) below)
+                if (C::V_STAGES >= 2 && has1) {
                     const int st = (n + 1) % C::V_STAGES;
                     if (n >= 1) ok = wait_warp(bar(C::BAR_VE + w * C::V_STAGES + st), ((n - 1) / C::V_STAGES) & 1, abort_flag);
                     if (!ok) break;
@@ -496,7 +536,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ptx::tc_fence_after();
                 issue_pv(n, j, 0);
                 ptx::mma_commit_elect(bar(C::BAR_OA + w));
-                if (j == 0) {
+                if (C::Q_BUFS >= 2 && j == 0) {
                     // First block of a tile: every Q K^T of the previous tile is
                     // complete (the softmax has seen S(n)), so its Q buffer takes
                     // the next tile's Q, which then lands during this tile.
@@ -516,10 +556,25 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (j == nkb - 1) ptx::mma_commit_elect(bar(C::BAR_PE + w));
                 if (!has1) break;
                 if (!issue_qk(n + 1, j1, 1, tnext)) { ok = false; break; }
+                if (C::V_STAGES == 1) {
+                    ok = wait_warp(bar(C::BAR_VE + w), n & 1, abort_flag);
+                    if (!ok) break;
+                    load_v(n + 1, L1, j1);
+                    ++v_loads;
+                }
                 // K(n+2) into the stage of K(n) (Q K^T(n) is complete: the softmax saw S(n))
                 if (has2) {
                     load_k(n + 2, L2, j2);
                     ++k_loads;
+                    if (C::Q_BUFS == 1 && j2 == 0) {
+                        // one Q buffer: the next tile's Q once Q K^T(n+1), the last
+                        // one of this tile, is done
+                        const int st = (n + 1) % C::K_STAGES;
+                        ok = wait_warp(bar(C::BAR_KE + w * C::K_STAGES + st), ((n + 1) / C::K_STAGES) & 1, abort_flag);
+                        if (!ok) break;
+                        load_q(L2, tnext + 1);
+                        ++q_loads;
+                    }
                 }
                 // V(n+1) to fp16
                 {
@@ -568,7 +623,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         int m_seen = 0;  // mask stages of this slice consumed
         bool ok = true;
         for (int it = 0, L = first_tile; L < p.num_tiles && ok; ++it, L += G) {
-            const TriTile t = tri_tile(p, L);
+            const TriTile t = tri_tile(p, L, C::NS);
             if (w >= t.nv) {
                 // No slice n0 + w in this tile: only release the shared bias tiles.
                 if (HAS_PAIR)
@@ -750,21 +805,21 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                                       : wait_half_b();
                                 if (!ready) { ok = false; break; }
                                 ptx::tc_fence_after();
-                                uint32_t o[D];
-                                if constexpr (D == 32) {
-                                    ptx::tmem_ld_x32(tO, o);
-                                    ptx::tmem_ld_wait_x32(o);
-                                } else {
-                                    ptx::tmem_ld_x16(tO, o);
-                                    ptx::tmem_ld_wait_x16(o);
-                                }
+                                constexpr int OCH = D < 32 ? D : 32;  // O columns per load
 #pragma unroll
-                                for (int e = 0; e < D; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                                if constexpr (D == 32) {
-                                    ptx::tmem_st_x16(tO, o);
-                                    ptx::tmem_st_x16(tO + 16, o + 16);
-                                } else {
-                                    ptx::tmem_st_x16(tO, o);
+                                for (int oc = 0; oc < D; oc += OCH) {
+                                    uint32_t o[OCH];
+                                    if constexpr (OCH == 32) {
+                                        ptx::tmem_ld_x32(tO + oc, o);
+                                        ptx::tmem_ld_wait_x32(o);
+                                    } else {
+                                        ptx::tmem_ld_x16(tO + oc, o);
+                                        ptx::tmem_ld_wait_x16(o);
+                                    }
+#pragma unroll
+                                    for (int e = 0; e < OCH; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+#pragma unroll
+                                    for (int e = 0; e < OCH; e += 16) ptx::tmem_st_x16(tO + oc + e, o + e);
                                 }
                             }
                         }
@@ -809,40 +864,50 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             ++tiles;
             if (!ok) break;
             ptx::tc_fence_after();
-            uint32_t o[D];
-            if constexpr (D == 32) {
-                ptx::tmem_ld_x32(tO, o);
-                ptx::tmem_ld_wait_x32(o);
-            } else {
-                ptx::tmem_ld_x16(tO, o);
-                ptx::tmem_ld_wait_x16(o);
-            }
             const float l = (suma.x + suma.y) + (sumb.x + sumb.y);
             const int n = t.n0 + w;
             const int row = t.qb * kBM + r;
-            if (row < p.S) {
+            {
                 const float inv_l = l > 0.f ? 1.f / l : 0.f;
                 bool finite = (l < INFINITY);  // an fp16 overflow of V shows up in O
                 uint16_t* orow = p.out + ((size_t(t.b) * p.N + n) * size_t(p.S) + size_t(row)) * size_t(p.H) * D +
                                  size_t(t.h) * D;
+                constexpr int OCH = D < 32 ? D : 32;  // O columns per load
+                // the tensor-memory loads are warp-collective: every lane takes
+                // them, only lanes with a row inside S store
 #pragma unroll
-                for (int k = 0; k < D; k += 8) {
-                    float f[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        f[e] = __uint_as_float(o[k + e]) * inv_l;
-                        finite = finite && fabsf(f[e]) < INFINITY;
+                for (int oc = 0; oc < D; oc += OCH) {
+                    uint32_t o[OCH];
+                    if constexpr (OCH == 32) {
+                        ptx::tmem_ld_x32(tO + oc, o);
+                        ptx::tmem_ld_wait_x32(o);
+                    } else {
+                        ptx::tmem_ld_x16(tO + oc, o);
+                        ptx::tmem_ld_wait_x16(o);
                     }
-                    uint4 v;
-                    v.x = ptx::pack_bf16x2(f[0], f[1]);
-                    v.y = ptx::pack_bf16x2(f[2], f[3]);
-                    v.z = ptx::pack_bf16x2(f[4], f[5]);
-                    v.w = ptx::pack_bf16x2(f[6], f[7]);
-                    *reinterpret_cast<uint4*>(orow + k) = v;
+                    if (row < p.S) {
+#pragma unroll
+                        for (int k = 0; k < OCH; k += 8) {
+                            float f[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                f[e] = __uint_as_float(o[k + e]) * inv_l;
+                                finite = finite && fabsf(f[e]) < INFINITY;
+                            }
+                            uint4 v;
+                            v.x = ptx::pack_bf16x2(f[0], f[1]);
+                            v.y = ptx::pack_bf16x2(f[2], f[3]);
+                            v.z = ptx::pack_bf16x2(f[4], f[5]);
+                            v.w = ptx::pack_bf16x2(f[6], f[7]);
+                            *reinterpret_cast<uint4*>(orow + oc + k) = v;
+                        }
+                    }
                 }
-                if (!finite) record_status(EVO_ERR_RANGE);
-                const float lse = l > 0.f ? (m + ptx::lg2_approx(l)) * kLn2 + c_cur : -INFINITY;
-                p.lse[((size_t(t.b) * p.N + n) * p.H + t.h) * size_t(p.S) + row] = lse;
+                if (row < p.S) {
+                    if (!finite) record_status(EVO_ERR_RANGE);
+                    const float lse = l > 0.f ? (m + ptx::lg2_approx(l)) * kLn2 + c_cur : -INFINITY;
+                    p.lse[((size_t(t.b) * p.N + n) * p.H + t.h) * size_t(p.S) + row] = lse;
+                }
             }
         }
         // on an abort, no tensor-memory access of this thread may still be in

@@ -167,6 +167,8 @@ __device__ __forceinline__ void mma_commit_elect(uint32_t bar) {
         : "memory");
 }
 
+// Arrives on the barrier with the expected byte count `bytes`, then loads
+// one box (the first box of a tile).
 __device__ __forceinline__ void tma_load_4d_elect(uint32_t dst, const CUtensorMap* m, uint32_t bar, uint32_t bytes,
                                                   int c0, int c1, int c2, int c3) {
     asm volatile(
@@ -176,6 +178,18 @@ __device__ __forceinline__ void tma_load_4d_elect(uint32_t dst, const CUtensorMa
         "@e cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3, %4, %5}], [%6];\n\t}" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar), "r"(bytes)
+        : "memory");
+}
+
+// Loads one more box of a tile whose barrier already expects its bytes.
+__device__ __forceinline__ void tma_load_4d_more_elect(uint32_t dst, const CUtensorMap* m, uint32_t bar, int c0,
+                                                       int c1, int c2, int c3) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];\n\t}" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
         : "memory");
 }
 

@@ -88,6 +88,8 @@ WORKLOADS = {
                          "large triangle attention, N_res=1024, D=32"),
     "tri_1024_d64": Workload("tri_1024_d64", 1, 1024, 1024, 4, 64, torch.bfloat16,
                              "large triangle attention, N_res=1024, D=64"),
+    "tri_512_d128": Workload("tri_512_d128", 1, 512, 512, 4, 128, torch.bfloat16,
+                             "triangle attention, N_res=512, D=128 (head-dim envelope)"),
 }
 
 
@@ -147,7 +149,7 @@ def make_case(name: str, seed: int = 0) -> Case:
         full = rng.choice(N, size=2, replace=False)
         keep[:, full, :] = False
         meta["fully_masked_n"] = sorted(int(x) for x in full)
-    elif name in ("tri_1024", "tri_1024_d64"):
+    elif name in ("tri_1024", "tri_1024_d64", "tri_512_d128"):
         pair = _normal(rng, (B, 1, H, S, S))
         spikes = rng.random((B, 1, H, S, S)) < 0.01
         pair[spikes] = np.float32(8.0)
