@@ -95,28 +95,21 @@ typedef enum {
  *   stream     CUDA stream the kernel is launched on.
  *
  * Supported envelope:
- *   EVO_DTYPE_BF16, tensor-core shapes: D in {16, 32, 64}, and with a pair
- *                   bias S a multiple of 8 (its rows are read by the
- *                   tensor-memory accelerator, which needs 16-byte row
- *                   strides).  Q, K, V, O, pair_bias 16-byte aligned;
- *                   mask_bias 2-byte aligned.  Runs on tcgen05 tensor cores
- *                   with fp32 accumulation in tensor memory.  The softmax
+ *   EVO_DTYPE_BF16, D in {16, 32, 64, 128}: the tcgen05 tensor-core kernel
+ *                   (fp32 accumulation in tensor memory; 3, 3, 2 and 1 n
+ *                   slices per tile).  Q, K, V, O 16-byte aligned;
+ *                   mask_bias 2-byte aligned; pair_bias 16-byte aligned when
+ *                   S is a multiple of 8 (its rows are then loaded by the
+ *                   tensor-memory accelerator), else 2-byte aligned (then
+ *                   read element by element, somewhat slower).  The softmax
  *                   numerators P are rounded to fp16 for the P.V product, so
  *                   V is converted to fp16 on chip: every |V| must be
  *                   <= 65504, else the kernel records EVO_ERR_RANGE (read by
  *                   evo_attn_sync_status) and O is not valid.
- *   EVO_DTYPE_BF16, other shapes: any other 1 <= D <= 128, or a pair bias
- *                   with S not a multiple of 8.  Every pointer 2-byte
- *                   aligned.  Runs on the SIMT kernel of EVO_DTYPE_FP32
- *                   (fp32 arithmetic from the exactly widened bf16 inputs, O
- *                   rounded to bf16), about 25 times slower than the
- *                   tensor-core shapes; no range limit on V.  A caller with
- *                   a pair bias and S not a multiple of 8 gets the same
- *                   result on the tensor-core kernel by padding S up to a
- *                   multiple of 8: padded keys carry a mask of -inf (so they
- *                   weigh exactly 0), padded Q/K/V/pair entries any finite
- *                   value, and the padded query rows of O and LSE are
- *                   discarded.
+ *   EVO_DTYPE_BF16, any other 1 <= D <= 128: the SIMT kernel of
+ *                   EVO_DTYPE_FP32 (fp32 arithmetic from the exactly widened
+ *                   bf16 inputs, O rounded to bf16), tens of times slower;
+ *                   every pointer 2-byte aligned; no range limit on V.
  *   EVO_DTYPE_FP32: 1 <= D <= 128, any S; 4-byte alignment.  Plain fp32 FMA.
  *   Every element count must fit in int64 and the grid in CUDA's limits.
  *   O and LSE must not overlap each other or any input.

@@ -82,9 +82,9 @@ def test_bf16_envelope(lib):
     # GPU that status marks an accepted shape.
     accepted = call()
     assert accepted == evo.EVO_ERR_INVALID_ARG
-    # head dims 16, 32, 64 and 128 go to the tensor-core kernel; other head
-    # dims up to 128, and pair biases whose rows are not whole 16-byte units,
-    # go to the SIMT kernel
+    # head dims 16, 32, 64 and 128 go to the tensor-core kernel (a pair bias
+    # whose rows are not whole 16-byte units read element by element); other
+    # head dims up to 128 go to the SIMT kernel
     for d in (1, 8, 24, 48, 64, 128):
         assert call(D=d) == accepted
     assert call(S=60, P=0x800000) == accepted

@@ -121,17 +121,34 @@ def test_bf16_random(shape):
     check_full(case, str(shape))
 
 
-# bf16 shapes outside the tensor-core kernel's envelope: the SIMT kernel with
-# bf16 inputs and output
+# bf16 head dims other than 16, 32, 64 and 128: the SIMT kernel with bf16
+# inputs and output
 BF16_SIMT_SHAPES = [
     # B, N, S, H, D, pair, mask, fully_masked
-    (1, 3, 70, 2, 128, True, "tail", 1),   # pair rows (S = 70) not 16-byte units
     (2, 2, 45, 3, 8, True, "tail", 0),     # small D, ragged S
     (1, 2, 130, 2, 48, False, "tail", 0),  # D not a multiple of 16
-    (1, 4, 60, 2, 32, True, "tail", 0),    # D = 32 with S % 8 != 0 and a pair bias
     (1, 2, 33, 1, 1, True, "zero", 0),     # D = 1
     (1, 2, 96, 2, 24, False, "neg_inf", 0),
 ]
+
+# tensor-core shapes whose pair-bias rows are not whole 16-byte units
+# (S % 8 != 0): the softmax reads the bias element by element from global
+# memory instead of through the TMA ring
+BF16_GLOBAL_BIAS_SHAPES = [
+    # B, N, S, H, D, pair, mask, fully_masked
+    (1, 3, 70, 2, 128, True, "tail", 1),   # D = 128, S < one tile
+    (1, 4, 60, 2, 32, True, "tail", 0),    # D = 32
+    (1, 5, 301, 2, 32, True, "bernoulli", 1),  # ragged, three key blocks, a fully masked n
+    (2, 3, 131, 1, 64, True, "head", 0),   # D = 64, two slices
+    (1, 2, 255, 2, 16, True, "none", 0),   # D = 16, no mask tensor (keys past S masked by the kernel)
+]
+
+
+@pytest.mark.parametrize("shape", BF16_GLOBAL_BIAS_SHAPES, ids=lambda s: "x".join(map(str, s[:5])) + f"-{s[6]}")
+def test_bf16_pair_bias_rows_not_16_byte_units(shape):
+    B, N, S, H, D, pair, mask, full = shape
+    case = W.random_case(B, N, S, H, D, torch.bfloat16, seed=6, mask=mask, pair=pair, fully_masked=full)
+    check_full(case, str(shape))
 
 
 @pytest.mark.parametrize("shape", BF16_SIMT_SHAPES, ids=lambda s: "x".join(map(str, s[:5])) + f"-{s[5]}-{s[6]}")

@@ -155,10 +155,14 @@ int launch_tri(int dev, const void* Q, const void* K, const void* V, const void*
     if (!encode_qkv(&tq, Q, B * N, S, H, D, C::SUBW) || !encode_qkv(&tk, K, B * N, S, H, D, C::SUBW) ||
         !encode_qkv(&tv, V, B * N, S, H, D, C::SUBW))
         return EVO_ERR_CUDA;
-    if (HAS_PAIR && !encode_pair(&tp, pair, B * H, S)) return EVO_ERR_CUDA;
+    // a pair bias whose rows are whole 16-byte units comes through the TMA
+    // ring; otherwise the softmax threads read it from global memory
+    const bool pair_tma = HAS_PAIR && S % 8 == 0;
+    if (pair_tma && !encode_pair(&tp, pair, B * H, S)) return EVO_ERR_CUDA;
 
     evo::TriParams p;
     p.mask = static_cast<const uint16_t*>(mask);
+    p.pair_g = (HAS_PAIR && !pair_tma) ? static_cast<const uint16_t*>(pair) : nullptr;
     p.out = static_cast<uint16_t*>(O);
     p.lse = LSE;
     p.N = int(N);
@@ -277,11 +281,9 @@ int check_fwd(const void* Q, const void* K, const void* V, const void* mask_bias
 
     if (!aligned(LSE, 4)) return EVO_ERR_MISALIGNED;
     const int64_t int_max = 2147483647;
-    // bf16 runs on the tensor-core kernel for D in {16, 32, 64} when the pair
-    // bias rows are whole 16-byte units (S a multiple of 8); every other bf16
-    // shape with D <= 128 runs on the SIMT kernel
-    *tensor_core = dtype == EVO_DTYPE_BF16 && (D == 16 || D == 32 || D == 64 || D == 128) &&
-                   !(pair_bias && (S % 8) != 0);
+    // bf16 runs on the tensor-core kernel for D in {16, 32, 64, 128}; every
+    // other bf16 head dim up to 128 runs on the SIMT kernel
+    *tensor_core = dtype == EVO_DTYPE_BF16 && (D == 16 || D == 32 || D == 64 || D == 128);
     if (*tensor_core) {
         // TMA coordinates are 32-bit; the CTA count (query blocks x heads x
         // n pairs x batch) must fit the grid's x dimension
@@ -290,8 +292,10 @@ int check_fwd(const void* Q, const void* K, const void* V, const void* mask_bias
             !mul_ok((S + evo::kBM - 1) / evo::kBM, bh, &ctas) ||
             !mul_ok(ctas, (N + evo::tri_slices(int(D)) - 1) / evo::tri_slices(int(D)), &ctas) || ctas > int_max)
             return EVO_ERR_UNSUPPORTED_SHAPE;
+        // the pair bias is loaded by TMA (16-byte rule) when S % 8 == 0, else
+        // element by element (2-byte rule)
         if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16) ||
-            (pair_bias && !aligned(pair_bias, 16)) || (mask_bias && !aligned(mask_bias, 2)))
+            (pair_bias && !aligned(pair_bias, S % 8 == 0 ? 16 : 2)) || (mask_bias && !aligned(mask_bias, 2)))
             return EVO_ERR_MISALIGNED;
     } else {
         if (D > evo::kF32MaxD) return EVO_ERR_UNSUPPORTED_SHAPE;

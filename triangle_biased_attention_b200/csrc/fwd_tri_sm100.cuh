@@ -59,6 +59,11 @@ namespace evo {
 
 struct TriParams {
     const uint16_t* mask;  // [B, N, S] bf16 bits, or nullptr
+    // [B, H, S, S] bf16 bits, read by the softmax threads straight from global
+    // memory, when its rows are not whole 16-byte units (S % 8 != 0) and the
+    // tensor-memory accelerator cannot load them; else nullptr (the bias
+    // tiles come through the TMA ring)
+    const uint16_t* pair_g;
     uint16_t* out;         // [B, N, S, H, D] bf16 bits
     float* lse;            // [B, N, H, S]
     int N, S, H;
@@ -267,9 +272,8 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             // through mc_s.  The mask values of the next block are fetched
             // from global memory before this block's are written, so their
             // latency overlaps a block.
-            if (lane == 0) {
-                ptx::prefetch_tmap(&tm_pair);
-            }
+            const bool bias_tma = HAS_PAIR && p.pair_g == nullptr;
+            if (bias_tma && lane == 0) ptx::prefetch_tmap(&tm_pair);
             int b_issued = 0, m_done[C::NS] = {};
             float c_run[C::NS];
 #pragma unroll
@@ -294,7 +298,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int it = 0, L = first_tile; L < p.num_tiles && ok; ++it, L += G) {
                 const TriTile t = tri_tile(p, L, C::NS);
                 for (int j = 0; j < nkb && ok; ++j) {
-                    if (HAS_PAIR) {
+                    if (bias_tma) {
                         const int st = b_issued % C::B_RING;
                         ok = wait_warp(bar(C::BAR_BE + st), ((b_issued / C::B_RING) & 1) ^ 1, abort_flag);
                         if (!ok) break;
@@ -361,7 +365,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                 }
             }
-            if (!ok && HAS_PAIR && lane == 0) {
+            if (!ok && bias_tma && lane == 0) {
                 // Let every bias copy this warp started land before the CTA exits.
                 for (int i2 = (b_issued > C::B_RING ? b_issued - C::B_RING : 0); i2 < b_issued; ++i2)
                     wait_bounded(bar(C::BAR_BF + i2 % C::B_RING), (i2 / C::B_RING) & 1, nullptr);
@@ -617,6 +621,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const float2 sqd2 = make_float2(p.sqrt_d, p.sqrt_d);
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
         const float inv_c = 1.0f / p.scale_log2;
+        const bool bias_tma = HAS_PAIR && p.pair_g == nullptr;
         int blk = 0;     // blocks of this slice processed (phase of SF / PF)
         int tiles = 0;   // tiles of this slice finished (phase of PE)
         int b_seen = 0;  // bias tiles consumed (every tile, valid slice or not)
@@ -626,7 +631,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const TriTile t = tri_tile(p, L, C::NS);
             if (w >= t.nv) {
                 // No slice n0 + w in this tile: only release the shared bias tiles.
-                if (HAS_PAIR)
+                if (bias_tma)
                     for (int j = 0; j < nkb && ok; ++j, ++b_seen) {
                         const int bs = b_seen % C::B_RING;
                         ok = wait_warp(bar(C::BAR_BF + bs), (b_seen / C::B_RING) & 1, abort_flag);
@@ -670,7 +675,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 const int bs = b_seen % C::B_RING;
                 uint32_t brow = 0;
-                if (HAS_PAIR) {
+                if (bias_tma) {
                     ok = wait_warp(bar(C::BAR_BF + bs), (b_seen / C::B_RING) & 1, abort_flag);
                     if (!ok) break;
                     brow = (sb + C::OFF_BIAS + uint32_t(bs * C::BIAS_BYTES) + uint32_t(r * 128)) |
@@ -678,13 +683,34 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     ++b_seen;
                 }
                 // bias words of a step (keys 32c .. 32c+31: 16 B groups 4c .. 4c+3 of the row)
+                // the row of pair bias this thread reads from global memory
+                // (S % 8 != 0); beyond S it reads nothing and adds 0 (those
+                // keys are -inf through the mask columns, those rows unused)
+                const uint16_t* grow = (HAS_PAIR && !bias_tma && t.qb * kBM + r < p.S)
+                                           ? p.pair_g + (size_t(t.b * p.H + t.h) * p.S + size_t(t.qb * kBM + r)) * p.S
+                                           : nullptr;
                 auto load_bias = [&](int c, uint4* bw) {
                     if (HAS_PAIR) {
+                        if (bias_tma) {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int g = 4 * c + q;
-                            bw[q] = ptx::ld_shared_v4((brow ^ uint32_t((g & 7) << 4)) +
-                                                      uint32_t((g >> 3) * (C::BIAS_BYTES / 2)));
+                            for (int q = 0; q < 4; ++q) {
+                                const int g = 4 * c + q;
+                                bw[q] = ptx::ld_shared_v4((brow ^ uint32_t((g & 7) << 4)) +
+                                                          uint32_t((g >> 3) * (C::BIAS_BYTES / 2)));
+                            }
+                        } else {
+                            uint32_t wds[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const int key = j * kBN + 32 * c + 2 * e;
+                                const uint32_t lo = (grow != nullptr && key < p.S) ? uint32_t(__ldg(grow + key)) : 0u;
+                                const uint32_t hi =
+                                    (grow != nullptr && key + 1 < p.S) ? uint32_t(__ldg(grow + key + 1)) : 0u;
+                                wds[e] = lo | (hi << 16);
+                            }
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                bw[q] = make_uint4(wds[4 * q], wds[4 * q + 1], wds[4 * q + 2], wds[4 * q + 3]);
                         }
                     }
                 };
@@ -749,7 +775,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                 for (int e = 0; e < 4; ++e)
                                     step_pair(4 * q + e, ptx::bf16lo_to_f32(wd[e]), ptx::bf16hi_to_f32(wd[e]));
                             }
-                            if (c == 3) ptx::mbar_arrive_elect(bar(C::BAR_BE + bs));
+                            if (bias_tma && c == 3) ptx::mbar_arrive_elect(bar(C::BAR_BE + bs));
                         } else {
 #pragma unroll
                             for (int e = 0; e < 16; ++e) step_pair(e, 0.f, 0.f);
