@@ -58,7 +58,8 @@ typedef struct CUstream_st* evo_stream_t;
 
 typedef enum {
     EVO_DTYPE_BF16 = 0,   /* bf16 inputs and O, fp32 arithmetic, tensor cores */
-    EVO_DTYPE_FP32 = 1    /* fp32 inputs and O, fp32 arithmetic throughout    */
+    EVO_DTYPE_FP32 = 1,   /* fp32 inputs and O, fp32 arithmetic throughout    */
+    EVO_DTYPE_FP16 = 2    /* fp16 inputs and O, as EVO_DTYPE_BF16              */
 } evo_dtype_t;
 
 typedef enum {
@@ -76,7 +77,7 @@ typedef enum {
 /*
  * evo_attn_fwd — the fused forward pass.
  *
- *   Q, K, V    [B, N, S, H, D] of `dtype`.
+ *   Q, K, V    [B, N, S, H, D] of `dtype` (bf16, fp16 or fp32).
  *   mask_bias  [B, N, 1, 1, S] of `dtype`, or NULL for no mask bias.  The
  *              guide's tests pass it as 1e9 * (mask - 1) (section 5.2), so a
  *              masked key carries -1e9 (-998244352 once rounded to bf16).  A
@@ -110,6 +111,12 @@ typedef enum {
  *                   EVO_DTYPE_FP32 (fp32 arithmetic from the exactly widened
  *                   bf16 inputs, O rounded to bf16), tens of times slower;
  *                   every pointer 2-byte aligned; no range limit on V.
+ *   EVO_DTYPE_FP16: the same envelope, kernels and alignment as
+ *                   EVO_DTYPE_BF16, with fp16 loads, biases and O (V needs
+ *                   no conversion).  The guide's mask 1e9 * (mask - 1) is
+ *                   -inf in fp16 (the guide notes fp16 for its own kernel,
+ *                   section 3.3), so a row whose every key is masked returns
+ *                   O = 0 and LSE = -inf.
  *   EVO_DTYPE_FP32: 1 <= D <= 128, any S; 4-byte alignment.  Plain fp32 FMA.
  *   Every element count must fit in int64 and the grid in CUDA's limits.
  *   O and LSE must not overlap each other or any input.

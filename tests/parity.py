@@ -1,6 +1,7 @@
 """Tolerances and comparison for GPU-vs-oracle parity.
 
-bf16 inputs (the stated bounds, applied as written):
+bf16 inputs, and fp16 inputs (held to the same bounds; their output
+spacing is finer) (the stated bounds, applied as written):
   * every element whose reference |O| < 4: |dO| <= 1e-2;
   * every element: the error of the arithmetic before the output is rounded
     to bf16 is at most 1e-2.  The kernel's fp32 value is not visible, only its
@@ -40,13 +41,14 @@ def _np(x):
     return np.asarray(x, dtype=np.float64)
 
 
-def half_spacing_bf16(x: np.ndarray) -> np.ndarray:
-    """Half the distance between neighbouring bf16 numbers at each bf16 value
-    x (8 significant bits): every real number that rounds to x lies within it
-    (for x a power of two, the spacing below is half as wide; the larger
-    one bounds both sides)."""
+def half_spacing_bf16(x: np.ndarray, bits: int = 8) -> np.ndarray:
+    """Half the distance between neighbouring numbers of a `bits`-significand
+    format (bf16: 8, fp16: 11) at each representable value x: every real
+    number that rounds to x lies within it (for x a power of two, the spacing
+    below is half as wide; the larger one bounds both sides).  Normal range
+    only (both formats' outputs here are far above their smallest normal)."""
     ax = np.maximum(np.abs(x), np.finfo(np.float32).tiny)
-    return np.exp2(np.floor(np.log2(ax)) - 8.0)
+    return np.exp2(np.floor(np.log2(ax)) - float(bits))
 
 
 def check(o_gpu, lse_gpu, o_ref, lse_ref, dtype, what=""):
@@ -61,8 +63,8 @@ def check(o_gpu, lse_gpu, o_ref, lse_ref, dtype, what=""):
     dL = np.abs(lse_gpu[fin] - lse_ref[fin])
     stats = {"max_dO": float(dO.max(initial=0)), "mean_dO": float(dO.mean()) if dO.size else 0.0,
              "max_dLSE": float(dL.max(initial=0)), "max_abs_O": float(np.abs(o_ref).max(initial=0))}
-    if dtype == torch.bfloat16:
-        half = half_spacing_bf16(o_gpu)
+    if dtype in (torch.bfloat16, torch.float16):
+        half = half_spacing_bf16(o_gpu, 8 if dtype == torch.bfloat16 else 11)
         stats["max_arith_err_lower_bound"] = float(np.maximum(dO - half, 0.0).max(initial=0))
         small = np.abs(o_ref) < BF16_STRICT_BELOW
         stats["max_dO_below_4"] = float(dO[small].max(initial=0))

@@ -63,7 +63,8 @@ def test_invalid_arguments(lib):
     assert call(B=-1) == evo.EVO_ERR_INVALID_ARG
     assert call(S=-5) == evo.EVO_ERR_INVALID_ARG
     assert call(dtype=7) == evo.EVO_ERR_UNSUPPORTED_DTYPE
-    assert call(dtype=2) == evo.EVO_ERR_UNSUPPORTED_DTYPE   # fp16 is not offered
+    assert call(dtype=3) == evo.EVO_ERR_UNSUPPORTED_DTYPE
+    assert call(dtype=evo.EVO_DTYPE_FP16) == call()         # fp16: the bf16 envelope
     assert call(D=0) == evo.EVO_ERR_UNSUPPORTED_SHAPE
 
 

@@ -224,3 +224,26 @@ def test_buffers_on_another_device_are_rejected():
                           1, 2, 128, 1, 32, evo.EVO_DTYPE_BF16, None)
     assert st == evo.EVO_ERR_INVALID_ARG
     assert torch.cuda.current_device() == before
+
+
+# fp16 inputs: the same kernels with fp16 loads, bias, mask and output (the
+# score MMA runs fp16 x fp16; V needs no conversion).  The guide's mask
+# 1e9 * (mask - 1) is -inf in fp16, so a fully masked n gives O = 0 and
+# LSE = -inf.
+FP16_SHAPES = [
+    # B, N, S, H, D, pair, mask, fully_masked, spike_frac
+    (1, 3, 200, 2, 32, True, "tail", 1, 0.0),
+    (1, 4, 256, 2, 64, True, "bernoulli", 0, 0.01),
+    (1, 2, 136, 1, 128, True, "head", 0, 0.0),
+    (1, 5, 60, 2, 16, True, "tail", 0, 0.0),      # S % 8 != 0: bias read element by element
+    (1, 3, 520, 2, 32, False, "neg_inf", 1, 0.0),  # no pair bias, five key blocks
+    (1, 2, 96, 2, 24, True, "tail", 1, 0.0),      # D = 24: the SIMT kernel
+]
+
+
+@pytest.mark.parametrize("shape", FP16_SHAPES, ids=lambda s: "x".join(map(str, s[:5])) + f"-{s[6]}")
+def test_fp16_random(shape):
+    B, N, S, H, D, pair, mask, full, spike = shape
+    case = W.random_case(B, N, S, H, D, torch.float16, seed=7, mask=mask, pair=pair,
+                         fully_masked=full, spike_frac=spike)
+    check_full(case, str(shape))

@@ -25,13 +25,14 @@ __all__ = [
     "evo_attn", "evo_attn_fwd", "evo_attn_sync_status", "evo_attn_strerror", "evo_attn_version",
     "evo_attn_selftest_timeout",
     "EvoAttnError", "library_path", "load_library",
-    "EVO_DTYPE_BF16", "EVO_DTYPE_FP32",
+    "EVO_DTYPE_BF16", "EVO_DTYPE_FP32", "EVO_DTYPE_FP16",
     "EVO_OK", "EVO_ERR_INVALID_ARG", "EVO_ERR_UNSUPPORTED_DTYPE", "EVO_ERR_UNSUPPORTED_SHAPE",
     "EVO_ERR_MISALIGNED", "EVO_ERR_CUDA", "EVO_ERR_TIMEOUT", "EVO_ERR_RANGE",
 ]
 
 EVO_DTYPE_BF16 = 0
 EVO_DTYPE_FP32 = 1
+EVO_DTYPE_FP16 = 2
 
 EVO_OK = 0
 EVO_ERR_INVALID_ARG = -1
@@ -46,7 +47,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libevoattn.so")
 _lib = None
 
-_DTYPES = {torch.bfloat16: EVO_DTYPE_BF16, torch.float32: EVO_DTYPE_FP32}
+_DTYPES = {torch.bfloat16: EVO_DTYPE_BF16, torch.float32: EVO_DTYPE_FP32, torch.float16: EVO_DTYPE_FP16}
 
 
 class EvoAttnError(RuntimeError):
@@ -127,7 +128,7 @@ def evo_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
              stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Biased-attention forward on CUDA tensors; returns (O, LSE).
 
-    q, k, v: [B, N, S, H, D] bf16 or fp32, contiguous, on one CUDA device.
+    q, k, v: [B, N, S, H, D] bf16, fp16 or fp32, contiguous, on one CUDA device.
     mask: [B, N, 1, 1, S] or None.  pair: [B, 1, H, S, S] or None (same dtype).
     out / lse: optional preallocated outputs ([B, N, S, H, D], [B, N, H, S] fp32).
     Runs on ``stream`` (default: the current stream) without synchronising.

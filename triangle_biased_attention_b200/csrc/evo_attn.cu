@@ -114,37 +114,39 @@ int select_device_of(const void* ptr, DeviceScope& scope) {
 // Q/K/V/O as a 4-D tensor {D, H, S, B*N}; a box is one (b, n, h) slice's
 // 128 rows of `box_w` elements (D, or 64 for D = 128, whose rows are loaded as
 // two boxes), swizzled over the box_w*2-byte row.
-bool encode_qkv(CUtensorMap* m, const void* base, int64_t BN, int64_t S, int64_t H, int64_t D, int64_t box_w) {
+bool encode_qkv(CUtensorMap* m, const void* base, int64_t BN, int64_t S, int64_t H, int64_t D, int64_t box_w,
+                CUtensorMapDataType dt) {
     const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(S), cuuint64_t(BN)};
     const cuuint64_t strides[3] = {cuuint64_t(D * 2), cuuint64_t(H * D * 2), cuuint64_t(S * H * D * 2)};
     const cuuint32_t box[4] = {cuuint32_t(box_w), 1, cuuint32_t(evo::kBM), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     const CUtensorMapSwizzle sw = box_w == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                               : (box_w == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
-    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+    return encode_fn()(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
                        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Pair bias as a 3-D tensor {S (key j), S (query i), B*H}; a box is 128
 // queries x 64 keys (128 B rows, 128 B swizzle).
-bool encode_pair(CUtensorMap* m, const void* base, int64_t BH, int64_t S) {
+bool encode_pair(CUtensorMap* m, const void* base, int64_t BH, int64_t S, CUtensorMapDataType dt) {
     const cuuint64_t dims[3] = {cuuint64_t(S), cuuint64_t(S), cuuint64_t(BH)};
     const cuuint64_t strides[2] = {cuuint64_t(S * 2), cuuint64_t(S * S * 2)};
     const cuuint32_t box[3] = {64, cuuint32_t(evo::kBM), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    return encode_fn()(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // The tcgen05 kernel: one CTA per SM, each walking the tiles (query block,
 // head, group of n slices, batch) with a stride of the grid size.
-template <int D, bool HAS_PAIR>
+template <int D, bool HAS_PAIR, bool F16>
 int launch_tri(int dev, const void* Q, const void* K, const void* V, const void* mask, const void* pair, void* O,
                float* LSE, int64_t B, int64_t N, int64_t S, int64_t H, cudaStream_t stream) {
-    using C = evo::TriCfg<D, HAS_PAIR>;
-    auto kernel = evo::evo_fwd_tri_kernel<D, HAS_PAIR>;
+    using C = evo::TriCfg<D, HAS_PAIR, F16>;
+    auto kernel = evo::evo_fwd_tri_kernel<D, HAS_PAIR, F16>;
+    const CUtensorMapDataType dt = F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     static AttrOnce attr;
     if (!attr.ensure(dev, kernel, C::SMEM_BYTES)) return EVO_ERR_CUDA;
     int sms = 0;
@@ -152,13 +154,13 @@ int launch_tri(int dev, const void* Q, const void* K, const void* V, const void*
         return EVO_ERR_CUDA;
     CUtensorMap tq, tk, tv, tp;
     std::memset(&tp, 0, sizeof(tp));
-    if (!encode_qkv(&tq, Q, B * N, S, H, D, C::SUBW) || !encode_qkv(&tk, K, B * N, S, H, D, C::SUBW) ||
-        !encode_qkv(&tv, V, B * N, S, H, D, C::SUBW))
+    if (!encode_qkv(&tq, Q, B * N, S, H, D, C::SUBW, dt) || !encode_qkv(&tk, K, B * N, S, H, D, C::SUBW, dt) ||
+        !encode_qkv(&tv, V, B * N, S, H, D, C::SUBW, dt))
         return EVO_ERR_CUDA;
     // a pair bias whose rows are whole 16-byte units comes through the TMA
     // ring; otherwise the softmax threads read it from global memory
     const bool pair_tma = HAS_PAIR && S % 8 == 0;
-    if (pair_tma && !encode_pair(&tp, pair, B * H, S)) return EVO_ERR_CUDA;
+    if (pair_tma && !encode_pair(&tp, pair, B * H, S, dt)) return EVO_ERR_CUDA;
 
     evo::TriParams p;
     p.mask = static_cast<const uint16_t*>(mask);
@@ -258,12 +260,12 @@ namespace {
 int check_fwd(const void* Q, const void* K, const void* V, const void* mask_bias, const void* pair_bias, void* O,
               float* LSE, int64_t B, int64_t N, int64_t S, int64_t H, int64_t D, int dtype, bool* tensor_core) {
     if (B < 0 || N < 0 || S < 0 || H < 0 || D < 0) return EVO_ERR_INVALID_ARG;
-    if (dtype != EVO_DTYPE_BF16 && dtype != EVO_DTYPE_FP32) return EVO_ERR_UNSUPPORTED_DTYPE;
+    if (dtype != EVO_DTYPE_BF16 && dtype != EVO_DTYPE_FP32 && dtype != EVO_DTYPE_FP16) return EVO_ERR_UNSUPPORTED_DTYPE;
     if (D == 0) return EVO_ERR_UNSUPPORTED_SHAPE;
     if (B == 0 || N == 0 || S == 0 || H == 0) return EVO_OK;  // nothing to compute
     if (!Q || !K || !V || !O || !LSE) return EVO_ERR_INVALID_ARG;
 
-    const int64_t es = dtype == EVO_DTYPE_BF16 ? 2 : 4;
+    const int64_t es = dtype == EVO_DTYPE_FP32 ? 4 : 2;
     int64_t bn, bns, bnsh, qkv_elems, qkv_bytes, mask_bytes, bh, pair_elems, pair_bytes, lse_bytes;
     if (!mul_ok(B, N, &bn) || !mul_ok(bn, S, &bns) || !mul_ok(bns, H, &bnsh) || !mul_ok(bnsh, D, &qkv_elems) ||
         !mul_ok(qkv_elems, es, &qkv_bytes) || !mul_ok(bns, es, &mask_bytes) || !mul_ok(B, H, &bh) ||
@@ -283,7 +285,7 @@ int check_fwd(const void* Q, const void* K, const void* V, const void* mask_bias
     const int64_t int_max = 2147483647;
     // bf16 runs on the tensor-core kernel for D in {16, 32, 64, 128}; every
     // other bf16 head dim up to 128 runs on the SIMT kernel
-    *tensor_core = dtype == EVO_DTYPE_BF16 && (D == 16 || D == 32 || D == 64 || D == 128);
+    *tensor_core = dtype != EVO_DTYPE_FP32 && (D == 16 || D == 32 || D == 64 || D == 128);
     if (*tensor_core) {
         // TMA coordinates are 32-bit; the CTA count (query blocks x heads x
         // n pairs x batch) must fit the grid's x dimension
@@ -318,13 +320,19 @@ int launch_fwd(int dev, bool tensor_core, const void* Q, const void* K, const vo
     if (dtype == EVO_DTYPE_FP32)
         return launch_f32<float>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, st);
     if (!tensor_core)
-        return launch_f32<uint16_t>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, st);
+        return dtype == EVO_DTYPE_FP16
+                   ? launch_f32<__half>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, st)
+                   : launch_f32<uint16_t>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, D, st);
 
     if (encode_fn() == nullptr) return EVO_ERR_CUDA;
     const bool has_pair = pair_bias != nullptr;
-#define EVO_LAUNCH_TRI(DD)                                                                            \
-    return has_pair ? launch_tri<DD, true>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st) \
-                    : launch_tri<DD, false>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st)
+    const bool f16 = dtype == EVO_DTYPE_FP16;
+#define EVO_LAUNCH_TRI(DD)                                                                                        \
+    if (f16)                                                                                                      \
+        return has_pair ? launch_tri<DD, true, true>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st)  \
+                        : launch_tri<DD, false, true>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st); \
+    return has_pair ? launch_tri<DD, true, false>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st)      \
+                    : launch_tri<DD, false, false>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, B, N, S, H, st)
     switch (D) {
         case 16: EVO_LAUNCH_TRI(16);
         case 32: EVO_LAUNCH_TRI(32);
@@ -440,7 +448,7 @@ extern "C" EVO_API const char* evo_attn_strerror(int status) {
         case EVO_ERR_MISALIGNED: return "a pointer breaks the alignment rule";
         case EVO_ERR_CUDA: return "a CUDA call failed";
         case EVO_ERR_TIMEOUT: return "a device-side wait timed out";
-        case EVO_ERR_RANGE: return "an input value is outside the supported range (|V| > 65504 with bf16)";
+        case EVO_ERR_RANGE: return "an input value is outside the supported range (|V| > 65504 with bf16, or a non-finite output)";
         default: return "unknown status";
     }
 }
@@ -462,7 +470,7 @@ extern "C" EVO_API int evo_attn_fwd_host(const void* Qh, const void* Kh, const v
     if (B == 0 || N == 0 || S == 0 || H == 0) return EVO_OK;
     if (!Qh || !Kh || !Vh || !Oh || !LSEh) return EVO_ERR_INVALID_ARG;
     RelaxedCapture relaxed;
-    const int64_t es = dtype == EVO_DTYPE_BF16 ? 2 : 4;
+    const int64_t es = dtype == EVO_DTYPE_FP32 ? 4 : 2;
     // sizes fit int64: check_fwd multiplied them out already
     const int64_t row = S * H * D * es;  // bytes of one (b, n) slice of Q, K, V or O
     const int64_t mrow = S * es, lrow = H * S * 4, prow = H * S * S * es;

@@ -17,6 +17,7 @@
 #include <cstdint>
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 
@@ -34,8 +35,11 @@ __device__ __forceinline__ void st_elem(float* p, size_t i, float x) { p[i] = x;
 __device__ __forceinline__ void st_elem(uint16_t* p, size_t i, float x) {
     p[i] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
+// fp16 (exact widening; output rounded to nearest even)
+__device__ __forceinline__ float ld_elem(const __half* p, size_t i) { return __half2float(p[i]); }
+__device__ __forceinline__ void st_elem(__half* p, size_t i, float x) { p[i] = __float2half_rn(x); }
 
-template <typename T>  // float, or uint16_t holding bf16
+template <typename T>  // float, uint16_t holding bf16, or __half
 struct F32Params {
     const T* q;
     const T* k;

@@ -84,7 +84,7 @@ constexpr float kTriRescaleThreshold = 15.0f;
 // buffer plus a D-column O accumulator.
 __host__ __device__ constexpr int tri_slices(int D) { return D <= 32 ? 3 : (D == 64 ? 2 : 1); }
 
-template <int D, bool HAS_PAIR>
+template <int D, bool HAS_PAIR, bool F16 = false>
 struct TriCfg {
     static_assert(D == 16 || D == 32 || D == 64 || D == 128, "head dim");
     static constexpr int NS = tri_slices(D);          // slices per tile
@@ -152,9 +152,11 @@ struct TriCfg {
     static constexpr uint32_t TMEM_COLS = (TM_O0 + NS * D) <= 256 ? 256u : 512u;
     static_assert(TM_O0 + NS * D <= TMEM_COLS, "tensor memory");
     // instruction descriptors, fp32 accumulate, M = 128
-    // Q K^T of one half block: bf16 x bf16, both K-major, N = 64 keys
-    static constexpr uint32_t IDESC_QK =
+    // Q K^T of one half block: bf16 x bf16 (or fp16 x fp16), both K-major,
+    // N = 64 keys; the mask step is always bf16 x bf16
+    static constexpr uint32_t IDESC_MASK =
         (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(kBN / 2) >> 3) << 17) | ((uint32_t(kBM) >> 4) << 24);
+    static constexpr uint32_t IDESC_QK = F16 ? (IDESC_MASK & ~((1u << 7) | (1u << 10))) : IDESC_MASK;
     static constexpr uint32_t IDESC_PV =
         (1u << 4) | (0u << 7) | (0u << 10) | (1u << 16) | ((uint32_t(D) >> 3) << 17) | ((uint32_t(kBM) >> 4) << 24);
 };
@@ -177,17 +179,42 @@ __device__ __forceinline__ TriTile tri_tile(const TriParams& p, int L, int ns) {
     return t;
 }
 
+// One 16-bit element (bf16 or fp16 bits) -> fp32, exact.
+template <bool F16>
+__device__ __forceinline__ float elem_to_f32(uint32_t bits) {
+    if constexpr (F16) return __half2float(__ushort_as_half(uint16_t(bits)));
+    else return __uint_as_float(bits << 16);
+}
+// A pair of 16-bit elements in one word (lower index in the low half) -> fp32 x 2.
+template <bool F16>
+__device__ __forceinline__ float2 pair_to_f32x2(uint32_t w) {
+    if constexpr (F16) {
+        const __half2 h = *reinterpret_cast<const __half2*>(&w);
+        return __half22float2(h);
+    } else {
+        return make_float2(ptx::bf16lo_to_f32(w), ptx::bf16hi_to_f32(w));
+    }
+}
+// Two fp32 -> the output type, round to nearest even; `lo` in the low half.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_out(float lo, float hi) {
+    if constexpr (F16) return ptx::pack_f16x2(lo, hi);
+    else return ptx::pack_bf16x2(lo, hi);
+}
+
 __device__ __forceinline__ void tmem_ld_x32f(uint32_t taddr, float* f) {
     ptx::tmem_ld_x32(taddr, reinterpret_cast<uint32_t*>(f));
 }
 __device__ __forceinline__ void tmem_wait_x32f(float* f) { ptx::tmem_ld_wait_x32(reinterpret_cast<uint32_t*>(f)); }
 
-template <int D, bool HAS_PAIR>
-__global__ void __launch_bounds__(TriCfg<D, HAS_PAIR>::THREADS, 1)
+// F16: Q, K, V, biases and O in fp16 instead of bf16 (V then needs no
+// conversion for the P.V product, which is fp16 x fp16 either way).
+template <int D, bool HAS_PAIR, bool F16>
+__global__ void __launch_bounds__(TriCfg<D, HAS_PAIR, F16>::THREADS, 1)
 evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_pair,
                    const TriParams p) {
-    using C = TriCfg<D, HAS_PAIR>;
+    using C = TriCfg<D, HAS_PAIR, F16>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = ptx::smem_u32(smem);
@@ -329,7 +356,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const int key = j * kBN + lane + 32 * k;
-                            v[k] = key < p.S ? __uint_as_float(cur[w][k] << 16) : -INFINITY;
+                            v[k] = key < p.S ? elem_to_f32<F16>(cur[w][k]) : -INFINITY;
                             bmax = fmaxf(bmax, v[k]);
                         }
 #pragma unroll
@@ -464,7 +491,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (aug)
                     ptx::mma_ss_elect(d, a_aug,
                                       desc_k_major<C::AUG_ROW>(sb + C::OFF_KAUG + ms * C::AUG_TILE + hf * 64 * C::AUG_ROW),
-                                      C::IDESC_QK, 1u);
+                                      C::IDESC_MASK, 1u);
                 if (hf == 1) {
                     if (aug) ptx::mma_commit_elect(bar(C::BAR_ME + ms));
                     ptx::mma_commit_elect(bar(C::BAR_KE + w * C::K_STAGES + st));
@@ -508,7 +535,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 load_v(0, L, 0);
                 ++v_loads;
                 ok = wait_warp(bar(C::BAR_VF + w * C::V_STAGES), 0, abort_flag);
-                if (ok) convert_v_chunks<0, C::V_CHUNKS, true>(v_tile(0), lane);
+                if (ok && !F16) convert_v_chunks<0, C::V_CHUNKS, true>(v_tile(0), lane);
                 ok = ok && issue_qk(0, 0, 0, 0) && issue_qk(0, 0, 1, 0);
                 if (ok && C::Q_BUFS == 1 && next_pos(L, 0, L1, j1) && j1 == 0) {
                     // one key block per tile and one Q buffer: position 1 needs the
@@ -585,7 +612,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     const int st = (n + 1) % C::V_STAGES;
                     ok = wait_warp(bar(C::BAR_VF + w * C::V_STAGES + st), ((n + 1) / C::V_STAGES) & 1, abort_flag);
                     if (!ok) break;
-                    convert_v_chunks<0, C::V_CHUNKS, true>(v_tile(st), lane);
+                    if (!F16) convert_v_chunks<0, C::V_CHUNKS, true>(v_tile(st), lane);
                 }
                 L = L1;
                 j = j1;
@@ -772,8 +799,10 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             for (int q = 0; q < 4; ++q) {
                                 const uint32_t wd[4] = {bw[q].x, bw[q].y, bw[q].z, bw[q].w};
 #pragma unroll
-                                for (int e = 0; e < 4; ++e)
-                                    step_pair(4 * q + e, ptx::bf16lo_to_f32(wd[e]), ptx::bf16hi_to_f32(wd[e]));
+                                for (int e = 0; e < 4; ++e) {
+                                    const float2 b = pair_to_f32x2<F16>(wd[e]);
+                                    step_pair(4 * q + e, b.x, b.y);
+                                }
                             }
                             if (bias_tma && c == 3) ptx::mbar_arrive_elect(bar(C::BAR_BE + bs));
                         } else {
@@ -921,10 +950,10 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                 finite = finite && fabsf(f[e]) < INFINITY;
                             }
                             uint4 v;
-                            v.x = ptx::pack_bf16x2(f[0], f[1]);
-                            v.y = ptx::pack_bf16x2(f[2], f[3]);
-                            v.z = ptx::pack_bf16x2(f[4], f[5]);
-                            v.w = ptx::pack_bf16x2(f[6], f[7]);
+                            v.x = pack_out<F16>(f[0], f[1]);
+                            v.y = pack_out<F16>(f[2], f[3]);
+                            v.z = pack_out<F16>(f[4], f[5]);
+                            v.w = pack_out<F16>(f[6], f[7]);
                             *reinterpret_cast<uint4*>(orow + oc + k) = v;
                         }
                     }
