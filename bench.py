@@ -50,9 +50,12 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="tri_1024", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=5,
+                    help="steps of the host-memory leg (0 skips it; e2e is then null)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="write a 256 MB buffer before every timed step and time the kernels alone (cold L2)")
     return ap.parse_args()
 
 
@@ -256,11 +259,24 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(wl):
+def workload_config(wl, flush=False):
     return {"workload": wl.name, "B": wl.B, "N": wl.N, "S": wl.S, "H": wl.H, "D": wl.D,
             "dtype": "bf16" if wl.dtype == torch.bfloat16 else "fp32",
-            "l2": "inputs (%.2f GB) larger than the 126 MB L2; no flush" % (alg_bytes(wl) / 1e9),
+            "l2": ("256 MB written before every step; kernels timed alone (cold L2)" if flush else
+                   "inputs (%.2f GB) %s the 126 MB L2; no flush" % (
+                       alg_bytes(wl) / 1e9, "larger than" if alg_bytes(wl) > 126e6 else "NOT larger than")),
             "parallelism": "replicas (one full workload per GPU)"}
+
+
+def pair_bias_stream(wl) -> int:
+    """Bytes of pair-bias tiles loaded per launch (0 without a pair bias, or
+    when S % 8 != 0 and the softmax reads the bias from global memory)."""
+    if wl.name == "msa_col_2048" or wl.dtype == torch.float32 or wl.S % 8:
+        return 0
+    ns = 3 if wl.D <= 32 else (2 if wl.D == 64 else 1)
+    qb = (wl.S + 127) // 128
+    tiles = qb * wl.H * ((wl.N + ns - 1) // ns) * wl.B
+    return tiles * qb * 128 * 128 * 2
 
 
 def alg_bytes(wl) -> int:
@@ -301,14 +317,31 @@ def run_ours(args, rank, world, local):
     sampler = ClockSampler(dev.index)
     barrier(world)
     torch.cuda.synchronize(dev)
-    with sampler:
-        start.record(stream)
-        for _ in range(args.steps):
-            step()
-        stop.record(stream)
-        torch.cuda.synchronize(dev)
-    barrier(world)
-    ms = start.elapsed_time(stop)
+    if args.flush_l2:
+        # cold L2: a 256 MB write (twice the 126 MB L2) before every step; only
+        # the kernels are timed, each between its own pair of events
+        scratch = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        with sampler:
+            for e0, e1 in evs:
+                with torch.cuda.stream(stream):
+                    scratch.fill_(1)
+                e0.record(stream)
+                step()
+                e1.record(stream)
+            torch.cuda.synchronize(dev)
+        barrier(world)
+        ms = sum(e0.elapsed_time(e1) for e0, e1 in evs)
+    else:
+        with sampler:
+            start.record(stream)
+            for _ in range(args.steps):
+                step()
+            stop.record(stream)
+            torch.cuda.synchronize(dev)
+        barrier(world)
+        ms = start.elapsed_time(stop)
     status = evo.evo_attn_sync_status(stream.cuda_stream)
     if status != evo.EVO_OK:
         raise RuntimeError(f"kernel status {status}: {evo.evo_attn_strerror(status)}")
@@ -329,20 +362,23 @@ def run_ours(args, rank, world, local):
     def e2e_step():
         evo.evo_attn_from_host(*host_in, out=host_o, lse=host_lse, device_buffers=dev_bufs, stream=stream)
 
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize(dev)
+    e2e = None
+    if args.e2e_steps > 0:
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                e2e_step()
+            torch.cuda.synchronize(dev)
+            barrier(world)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.e2e_steps):
+                e2e_step()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
         barrier(world)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.e2e_steps
-    e2e_value = world * flops / (e2e_ms * 1e-3) / 1e12
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / args.e2e_steps
+        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": args.e2e_steps}
 
     peaks, peak_src = load_peaks()
     achieved = flops / (ms / args.steps * 1e-3) / 1e12  # this rank's kernel, per launch
@@ -361,6 +397,13 @@ def run_ours(args, rank, world, local):
         else "fallback (6.65 TB/s, 1.59 PFLOP/s)"
     roof["alg_flops_per_launch"] = flops
     roof["alg_bytes_per_launch"] = alg_bytes(wl)
+    bias = pair_bias_stream(wl)
+    if bias:
+        # the pair-bias tiles the kernel moves from L2 into shared memory: one
+        # 128 x 128 tile per (tile, key block), shared by the slices of a tile
+        roof["pair_bias_stream"] = {"l2_to_sm_bytes_per_launch": bias,
+                                    "gbs": bias / (ms / args.steps * 1e-3) / 1e9,
+                                    "unique_bytes": wl.B * wl.H * wl.S * wl.S * 2}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -372,12 +415,11 @@ def run_ours(args, rank, world, local):
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic (seeded numpy PCG64, bf16)",
-            "config": workload_config(wl),
+            "config": workload_config(wl, args.flush_l2),
             "roofline_pct": 100.0 * roof["frac"] if bound == "tensor" else 100.0 * roof["frac"],
             "roofline": roof,
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms, "steps": args.e2e_steps},
+            "e2e": e2e,
             "gpu_launches": args.steps,
             "kernel": KERNEL_NAME,
             "clocks": sampler.record(),
