@@ -1,6 +1,6 @@
 /*
- * evo_attn.h — C ABI of the B200 (sm_100a) biased-attention forward library,
- * libevoattn.so.
+ * evo_attn.h — C ABI of the B200 (sm_100a) biased-attention library,
+ * libevoattn.so: the forward pass and its backward pass.
  *
  * The operation is the forward pass that the DeepSpeed DS4Sci_EvoformerAttention
  * guide (hmyw.cn) describes for the four Evoformer attention variants (its
@@ -169,6 +169,72 @@ EVO_API int evo_attn_fwd_host(const void* Qh, const void* Kh, const void* Vh, co
                       void* Qd, void* Kd, void* Vd, void* mask_d, void* pair_d, void* Od, float* LSEd,
                       int64_t B, int64_t N, int64_t S, int64_t H, int64_t D, int dtype, int64_t chunk_n,
                       evo_stream_t stream);
+
+/*
+ * evo_attn_bwd_workspace_size — bytes of device workspace evo_attn_bwd needs
+ * for these sizes (the same for every dtype and for every choice of
+ * requested bias gradients), or a negative evo_status_t for negative sizes
+ * (EVO_ERR_INVALID_ARG) or sizes whose byte counts overflow int64
+ * (EVO_ERR_UNSUPPORTED_SHAPE).
+ */
+EVO_API int64_t evo_attn_bwd_workspace_size(int64_t B, int64_t N, int64_t S, int64_t H, int64_t D);
+
+/*
+ * evo_attn_bwd — the backward pass: gradients of a loss with respect to the
+ * inputs of evo_attn_fwd, given the gradient dO with respect to O.
+ *
+ * The guide (sections 1 and 5.4) describes the backward kernel of its
+ * FlashAttention-style design: it does not keep the S x S attention weights
+ * of the forward pass but recomputes them from Q, K, V, O and the forward's
+ * log-sum-exp, with the per-row delta = dO . O as an intermediate, and it
+ * computes the gradient of a bias only when the caller needs it.  The guide
+ * gives no formula; the gradients are the chain rule of the forward formula
+ * above.  Per (b, n, h) slice, with p_ij the softmax weights and
+ * dt_ij = p_ij (dO_i . V_j - delta_i) the gradient of the logit t_ij:
+ *     dQ_i = sum_j dt_ij K_j / sqrt(D),   dK_j = sum_i dt_ij Q_i / sqrt(D),
+ *     dV_j = sum_i p_ij dO_i,
+ *     dmask[b,n,0,0,j] = sum_h sum_i dt_ij    (the mask is shared by heads and rows),
+ *     dpair[b,0,h,i,j] = sum_n dt_ij          (the pair bias is shared by every n).
+ *
+ *   Q, K, V, mask_bias, pair_bias, dtype, B, N, S, H, D
+ *              as passed to evo_attn_fwd (same layouts and NULL rules).
+ *   O, LSE     the outputs of evo_attn_fwd for exactly those inputs.
+ *   dO         [B, N, S, H, D] of `dtype`: the gradient with respect to O.
+ *   dQ, dK, dV [B, N, S, H, D] of `dtype`, written.
+ *   dmask      [B, N, 1, 1, S] of `dtype`, written, or NULL to skip this
+ *              gradient (NULL is required when mask_bias is NULL).
+ *   dpair      [B, 1, H, S, S] of `dtype`, written, or NULL to skip this
+ *              gradient (NULL is required when pair_bias is NULL).
+ *   workspace  device scratch of at least evo_attn_bwd_workspace_size(B, N,
+ *              S, H, D) bytes (workspace_bytes says how many), 256-byte
+ *              aligned, owned by the caller; its contents on entry do not
+ *              matter and are overwritten.  Keep it allocated and do not use
+ *              it for anything else until the call's work on `stream` is done.
+ *   stream     CUDA stream the kernels are launched on.
+ *
+ * A row whose every key carries the guide's -1e9 mask follows the formula
+ * (the mask is a constant shift of the row, as in the forward pass); its
+ * row statistics are then recomputed from the inputs, because the fp32 LSE
+ * near -1e9 has lost the digits that matter.  A row with no finite logit
+ * (every key -inf) has no weights and contributes zero to every gradient.
+ *
+ * Supported envelope: every dtype, 1 <= D <= 128, any S, with plain fp32
+ * FMA arithmetic (recomputing the weights per gradient); pointers aligned to
+ * the element size (LSE to 4 bytes).  The gradients of a call are computed
+ * by several kernels on `stream` and are complete once its work there is.
+ * Outputs and workspace must not overlap each other or any input.
+ *
+ * Returns EVO_OK once the work is enqueued, or a negative evo_status_t
+ * (EVO_ERR_INVALID_ARG also for a workspace that is too small, or a gradient
+ * of a bias that was not passed).
+ */
+EVO_API int evo_attn_bwd(const void* Q, const void* K, const void* V,
+                 const void* mask_bias, const void* pair_bias,
+                 const void* O, const float* LSE, const void* dO,
+                 void* dQ, void* dK, void* dV, void* dmask, void* dpair,
+                 void* workspace, int64_t workspace_bytes,
+                 int64_t B, int64_t N, int64_t S, int64_t H, int64_t D,
+                 int dtype, evo_stream_t stream);
 
 /*
  * evo_attn_sync_status — synchronise `stream`, then return and clear the

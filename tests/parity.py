@@ -82,3 +82,44 @@ def check(o_gpu, lse_gpu, o_ref, lse_ref, dtype, what=""):
         assert stats["max_dO"] <= FP32_REL * scale, f"{what}: {stats}"
         assert np.all(dL <= FP32_REL * np.maximum(1.0, np.abs(lse_ref[fin]))), f"{what}: LSE {stats}"
     return stats
+
+
+# Backward pass.  The gradients are sums over many products whose factors the
+# tensor-core path rounds to bf16 (weights p, logit gradients dt; O enters
+# delta after its own rounding) before it accumulates in fp32, and the
+# gradients are rounded to the input dtype at the end: each source moves a
+# gradient by up to about 2^-9 of the size of its terms.  Held normwise per
+# gradient tensor G against the float64 reference R:
+#   bf16 / fp16:  max |G - R| <= 2^-6 max |R|  and  mean |G - R| <= 2^-7 mean |R|
+#                 (eight and four times the 2^-9 rounding unit);
+#   fp32:         max |G - R| <= 1e-5 max |R|  (the forward's normwise reading).
+BWD_MAX_REL = 2.0 ** -6
+BWD_MEAN_REL = 2.0 ** -7
+BWD_FP32_MAX_REL = 1e-5
+
+
+def check_grads(got: dict, ref: dict, dtype, what=""):
+    stats = {}
+    for name, r in ref.items():
+        g = got[name]
+        assert g is not None, f"{what}: {name} not computed"
+        g, r = _np(g), _np(r)
+        assert g.shape == r.shape, f"{what}: {name} shape {g.shape} vs {r.shape}"
+        assert np.all(np.isfinite(g)), f"{what}: non-finite {name}"
+        e = np.abs(g - r)
+        rmax = float(np.abs(r).max(initial=0))
+        rmean = float(np.abs(r).mean()) if r.size else 0.0
+        s = {"max_err": float(e.max(initial=0)), "max_ref": rmax,
+             "max_rel": float(e.max(initial=0)) / max(rmax, 1e-30),
+             "mean_rel": (float(e.mean()) / max(rmean, 1e-30)) if e.size else 0.0}
+        stats[name] = s
+        if dtype in (torch.bfloat16, torch.float16):
+            ok = s["max_err"] <= BWD_MAX_REL * rmax and float(e.mean()) <= BWD_MEAN_REL * rmean
+        else:
+            ok = s["max_err"] <= BWD_FP32_MAX_REL * rmax
+        if rmax == 0.0:
+            ok = s["max_err"] == 0.0
+        assert ok, f"{what}: {name} {s}"
+    print(f"grad parity {what}: " + ", ".join(
+        f"{k} max_rel {v['max_rel']:.2e} mean_rel {v['mean_rel']:.2e}" for k, v in stats.items()))
+    return stats

@@ -172,3 +172,70 @@ def test_host_entry_checks_arguments(lib):
     assert call_host(dtype=7) == evo.EVO_ERR_UNSUPPORTED_DTYPE
     # made-up host addresses are not page-locked memory
     assert call_host() == evo.EVO_ERR_INVALID_ARG
+
+
+def call_bwd(M=None, P=None, dM=None, dP=None, W=0x10000000, Wbytes=None, **kw):
+    """evo_attn_bwd with made-up device addresses (far apart, so nothing overlaps)."""
+    d = dict(B=1, N=2, S=64, H=2, D=32, dtype=evo.EVO_DTYPE_BF16)
+    d.update(kw)
+    if Wbytes is None:
+        Wbytes = max(evo.evo_attn_bwd_workspace_size(d["B"], d["N"], d["S"], d["H"], d["D"]), 0)
+    a = [0x1000000 * (i + 1) for i in range(9)]  # Q K V O LSE dO dQ dK dV
+    for key in ("Q", "K", "V", "O", "L", "dO", "dQ", "dK", "dV"):
+        if key in kw:
+            a["Q K V O L dO dQ dK dV".split().index(key)] = kw.pop(key)
+    return evo.evo_attn_bwd(a[0], a[1], a[2], M, P, a[3], a[4], a[5], a[6], a[7], a[8], dM, dP, W, Wbytes,
+                            d["B"], d["N"], d["S"], d["H"], d["D"], d["dtype"], None)
+
+
+def test_bwd_workspace_size(lib):
+    B, N, S, H, D = 1, 2, 64, 2, 32
+    size = evo.evo_attn_bwd_workspace_size(B, N, S, H, D)
+    r = lambda b: (b + 255) // 256 * 256
+    expect = (r(4 * B * N) + 2 * r(4 * B * N * H * S) + r(4 * B * N * S * H * D) + r(4 * B * N * S)
+              + r(4 * B * H * S * S))
+    assert size == expect
+    assert evo.evo_attn_bwd_workspace_size(-1, N, S, H, D) == evo.EVO_ERR_INVALID_ARG
+    assert evo.evo_attn_bwd_workspace_size(1 << 40, 1 << 40, S, H, D) == evo.EVO_ERR_UNSUPPORTED_SHAPE
+
+
+def test_bwd_checks_arguments(lib):
+    accepted = call_bwd()          # passes every check, then the made-up pointers are refused
+    assert accepted == evo.EVO_ERR_INVALID_ARG
+    # (a rejected argument gives another status, or the same one earlier:
+    # overlap tests below use addresses that pass every other check)
+    assert call_bwd(W=0x10000010) != accepted
+    assert call_bwd(B=0, W=None, Wbytes=0) == evo.EVO_OK
+    assert call_bwd(dtype=9) == evo.EVO_ERR_UNSUPPORTED_DTYPE
+    assert call_bwd(D=129) == evo.EVO_ERR_UNSUPPORTED_SHAPE
+    assert call_bwd(D=0) == evo.EVO_ERR_UNSUPPORTED_SHAPE
+    assert call_bwd(W=None) == evo.EVO_ERR_INVALID_ARG
+    # a workspace one byte short, or not on a 256-byte boundary
+    full = evo.evo_attn_bwd_workspace_size(1, 2, 64, 2, 32)
+    assert call_bwd(Wbytes=full - 1) == evo.EVO_ERR_INVALID_ARG
+    assert call_bwd(W=0x10000010) == evo.EVO_ERR_MISALIGNED
+    # a bias gradient needs its bias
+    assert call_bwd(dM=0xA000000) == evo.EVO_ERR_INVALID_ARG
+    assert call_bwd(dP=0xB000000) == evo.EVO_ERR_INVALID_ARG
+    assert call_bwd(M=0xC000000, dM=0xA000000, P=0xD000000, dP=0xB000000) == accepted
+    # outputs must not overlap inputs, each other or the workspace
+    assert call_bwd(dQ=0x1000000 + 64) == evo.EVO_ERR_INVALID_ARG         # dQ inside Q
+    assert call_bwd(dK=0x7000000 + 2) == evo.EVO_ERR_INVALID_ARG          # dK inside dQ
+    assert call_bwd(W=0x9000000 - 256) == evo.EVO_ERR_INVALID_ARG         # workspace runs into dV
+    # alignment to the element size
+    assert call_bwd(dV=0x9000001) == evo.EVO_ERR_MISALIGNED
+    assert call_bwd(L=0x5000002) == evo.EVO_ERR_MISALIGNED
+    assert call_bwd(dtype=evo.EVO_DTYPE_FP32, dO=0x6000002) == evo.EVO_ERR_MISALIGNED
+    assert call_bwd(D=48) == accepted and call_bwd(dtype=evo.EVO_DTYPE_FP32) == accepted
+
+
+def test_backward_wrapper_validates_before_calling():
+    import torch
+    q = torch.zeros(1, 2, 8, 1, 16)
+    lse = torch.zeros(1, 2, 1, 8)
+    with pytest.raises(ValueError):
+        evo.evo_attn_backward(q, q, q, None, None, q, lse, q)        # CPU tensors are refused
+    with pytest.raises(ValueError, match="without a mask"):
+        evo.evo_attn_backward(q, q, q, None, None, q, lse, q, need_dmask=True)
+    with pytest.raises(TypeError):
+        evo.evo_attn_backward(q, q, q, None, None, q, lse.double(), q)

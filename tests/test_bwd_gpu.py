@@ -1,0 +1,119 @@
+"""Backward pass on the GPU against the float64 oracle's gradients.
+
+Each case runs the forward pass (evo_attn) and then the backward pass
+(evo_attn_backward) through the C ABI on seeded inputs, and compares dQ, dK,
+dV and the requested bias gradients with the oracle's chain-rule gradients
+of the same inputs and upstream gradient, with the tolerances stated in
+tests/parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import triangle_biased_attention_b200 as evo
+from triangle_biased_attention_b200 import workloads as W
+from tests.parity import check_grads
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev():
+    return torch.device("cuda", 0)
+
+
+def _upstream(case, seed):
+    rng = np.random.Generator(np.random.PCG64(50_000 + seed))
+    return torch.from_numpy(rng.standard_normal(case.q.shape, dtype=np.float32)).to(case.q.dtype)
+
+
+def run_bwd(case, do, need_dmask=None, need_dpair=None):
+    dev = _dev()
+    to = (lambda t: None if t is None else t.to(dev))
+    q, k, v, m, p = to(case.q), to(case.k), to(case.v), to(case.mask), to(case.pair)
+    o, lse = evo.evo_attn(q, k, v, m, p)
+    grads = evo.evo_attn_backward(q, k, v, m, p, o, lse, to(do), need_dmask=need_dmask, need_dpair=need_dpair)
+    status = evo.evo_attn_sync_status()
+    assert status == evo.EVO_OK, evo.evo_attn_strerror(status)
+    names = ("dq", "dk", "dv", "dmask", "dpair")
+    return {n: (None if g is None else g.cpu()) for n, g in zip(names, grads)}
+
+
+def ref_grads(case, do):
+    return oracle.attention_bwd(case.q, case.k, case.v, case.mask, case.pair, do)
+
+
+def compare(case, seed, what, need_dmask=None, need_dpair=None):
+    do = _upstream(case, seed)
+    got = run_bwd(case, do, need_dmask, need_dpair)
+    ref = ref_grads(case, do)
+    if need_dmask is False:
+        assert got["dmask"] is None
+        ref.pop("dmask", None)
+    if need_dpair is False:
+        assert got["dpair"] is None
+        ref.pop("dpair", None)
+    return check_grads(got, ref, case.dtype, what)
+
+
+def test_bwd_tiny_fp32():
+    case = W.make_case("tiny_fp32", 0)
+    compare(case, 0, "tiny_fp32")
+
+
+# (B, N, S, H, D, mask, pair, spike_frac, fully_masked)
+BF16_CASES = [
+    (1, 4, 200, 2, 32, "tail", True, 0.01, 1),
+    (1, 3, 130, 2, 64, "head", True, 0.0, 0),
+    (2, 3, 96, 3, 16, "bernoulli", False, 0.0, 0),
+    (1, 2, 77, 2, 48, "tail", True, 0.0, 0),
+    (1, 3, 160, 2, 32, "neg_inf", True, 0.0, 0),
+    (1, 2, 64, 2, 32, "none", True, 0.0, 0),
+    (1, 1, 1, 1, 32, "zero", True, 0.0, 0),
+]
+
+
+@pytest.mark.parametrize("shape", BF16_CASES, ids=lambda s: "x".join(map(str, s[:5])) + f"-{s[5]}")
+def test_bwd_bf16(shape):
+    B, N, S, H, D, mask, pair, spike, full = shape
+    case = W.random_case(B, N, S, H, D, torch.bfloat16, seed=S + D, mask=mask, pair=pair, spike_frac=spike,
+                         fully_masked=full)
+    compare(case, S, f"bf16 {shape}")
+
+
+def test_bwd_fp32_random():
+    case = W.random_case(2, 3, 77, 2, 24, torch.float32, seed=5, mask="tail", pair=True, fully_masked=1)
+    compare(case, 5, "fp32 random")
+
+
+def test_bwd_fp16_fully_masked_rows_are_empty():
+    # in fp16 the guide's -1e9 mask is -inf: a fully masked n has no softmax
+    # and gets zero gradients
+    case = W.random_case(1, 3, 120, 2, 32, torch.float16, seed=6, mask="tail", pair=True, fully_masked=1)
+    stats = compare(case, 6, "fp16 with an empty n")
+    assert stats["dq"]["max_ref"] > 0
+
+
+def test_bwd_skips_bias_gradients_not_requested():
+    case = W.random_case(1, 2, 64, 2, 32, torch.bfloat16, seed=7, mask="tail", pair=True)
+    compare(case, 7, "no dmask", need_dmask=False)
+    compare(case, 7, "no dpair", need_dpair=False)
+
+
+def test_bwd_rejects_overlapping_outputs_on_device():
+    dev = _dev()
+    case = W.random_case(1, 2, 64, 2, 32, torch.bfloat16, seed=8, mask="none", pair=False)
+    q, k, v = (t.to(dev) for t in (case.q, case.k, case.v))
+    o, lse = evo.evo_attn(q, k, v)
+    do = torch.ones_like(q)
+    B, N, S, H, D = q.shape
+    size = evo.evo_attn_bwd_workspace_size(B, N, S, H, D)
+    ws = torch.empty(size, dtype=torch.uint8, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    args = lambda dq_ptr: (q.data_ptr(), k.data_ptr(), v.data_ptr(), None, None, o.data_ptr(), lse.data_ptr(),
+                           do.data_ptr(), dq_ptr, dk.data_ptr(), dv.data_ptr(), None, None, ws.data_ptr(), size,
+                           B, N, S, H, D, evo.EVO_DTYPE_BF16, None)
+    assert evo.evo_attn_bwd(*args(q.data_ptr())) == evo.EVO_ERR_INVALID_ARG     # dQ over Q
+    assert evo.evo_attn_bwd(*args(dk.data_ptr())) == evo.EVO_ERR_INVALID_ARG    # dQ over dK
+    assert evo.evo_attn_bwd(*args(dq.data_ptr())) == evo.EVO_OK
+    assert evo.evo_attn_sync_status() == evo.EVO_OK

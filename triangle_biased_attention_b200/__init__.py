@@ -1,4 +1,4 @@
-"""B200-native biased (Evoformer / Pairformer / triangle) attention forward.
+"""B200-native biased (Evoformer / Pairformer / triangle) attention.
 
 The computation is the forward pass of the DeepSpeed DS4Sci_EvoformerAttention
 guide (hmyw.cn, sections 4, 5.2-5.4):
@@ -7,7 +7,8 @@ guide (hmyw.cn, sections 4, 5.2-5.4):
     LSE = log sum exp of the same logits (natural log, fp32)
 
 with Q, K, V, O of shape [B, N, S, H, D], mask_bias [B, N, 1, 1, S] and
-pair_bias [B, 1, H, S, S] (shared by every n).  All arithmetic runs in the
+pair_bias [B, 1, H, S, S] (shared by every n), and its backward pass (the
+gradients of Q, K, V and of the biases, sections 1 and 5.4).  All arithmetic runs in the
 CUDA library ``libevoattn.so`` (hand-written sm_100a kernels behind the C ABI
 in ``include/evo_attn.h``); this module only marshals arguments through
 ctypes.  PyTorch supplies device memory and the current stream.  There is no
@@ -23,7 +24,7 @@ import torch
 
 __all__ = [
     "evo_attn", "evo_attn_fwd", "evo_attn_sync_status", "evo_attn_strerror", "evo_attn_version",
-    "evo_attn_selftest_timeout",
+    "evo_attn_selftest_timeout", "evo_attn_bwd", "evo_attn_bwd_workspace_size", "evo_attn_backward",
     "EvoAttnError", "library_path", "load_library",
     "EVO_DTYPE_BF16", "EVO_DTYPE_FP32", "EVO_DTYPE_FP16",
     "EVO_OK", "EVO_ERR_INVALID_ARG", "EVO_ERR_UNSUPPORTED_DTYPE", "EVO_ERR_UNSUPPORTED_SHAPE",
@@ -83,6 +84,10 @@ def load_library():
     lib.evo_attn_version.restype = i32
     lib.evo_attn_selftest_timeout.argtypes = [i64, vp, vp]
     lib.evo_attn_selftest_timeout.restype = i32
+    lib.evo_attn_bwd_workspace_size.argtypes = [i64, i64, i64, i64, i64]
+    lib.evo_attn_bwd_workspace_size.restype = i64
+    lib.evo_attn_bwd.argtypes = [vp] * 14 + [i64, i64, i64, i64, i64, i64, i32, vp]
+    lib.evo_attn_bwd.restype = i32
     _lib = lib
     return lib
 
@@ -116,6 +121,19 @@ def evo_attn_version() -> int:
 def evo_attn_selftest_timeout(limit_ns: int, result_ptr: int, stream: Optional[int] = None) -> int:
     """Launch the bounded-wait self-test (see include/evo_attn.h); returns the status code."""
     return int(load_library().evo_attn_selftest_timeout(limit_ns, result_ptr, stream))
+
+
+def evo_attn_bwd_workspace_size(B: int, N: int, S: int, H: int, D: int) -> int:
+    """Workspace bytes of evo_attn_bwd, or a negative status code."""
+    return int(load_library().evo_attn_bwd_workspace_size(B, N, S, H, D))
+
+
+def evo_attn_bwd(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair, workspace,
+                 workspace_bytes: int, B: int, N: int, S: int, H: int, D: int, dtype: int,
+                 stream: Optional[int]) -> int:
+    """The C backward entry point with raw addresses (ints); returns the status code."""
+    return int(load_library().evo_attn_bwd(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair,
+                                           workspace, workspace_bytes, B, N, S, H, D, dtype, stream))
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -230,3 +248,66 @@ def evo_attn_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         raise EvoAttnError(status, "evo_attn_fwd_host")
     out._evo_keepalive = (q, k, v, mask, pair, device_buffers)
     return out, lse
+
+
+def evo_attn_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                      mask: Optional[torch.Tensor], pair: Optional[torch.Tensor],
+                      o: torch.Tensor, lse: torch.Tensor, do: torch.Tensor,
+                      need_dmask: Optional[bool] = None, need_dpair: Optional[bool] = None,
+                      workspace: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None):
+    """Backward pass on CUDA tensors; returns (dq, dk, dv, dmask, dpair).
+
+    q, k, v, mask, pair: the forward's inputs; o, lse: its outputs (from
+    ``evo_attn``); do: the gradient with respect to o ([B, N, S, H, D], q's
+    dtype).  dmask ([B, N, 1, 1, S]) is computed when ``need_dmask`` (default:
+    a mask was passed), dpair ([B, 1, H, S, S]) when ``need_dpair`` (default:
+    a pair bias was passed); a gradient not computed comes back as None.
+    ``workspace``: an optional uint8 CUDA tensor of at least
+    ``evo_attn_bwd_workspace_size`` bytes (allocated here when not given).
+    Runs on ``stream`` (default: the current stream) without synchronising.
+    """
+    if q.dim() != 5:
+        raise ValueError("q must be [B, N, S, H, D]")
+    B, N, S, H, D = q.shape
+    if q.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {q.dtype}")
+    need_dmask = (mask is not None) if need_dmask is None else bool(need_dmask)
+    need_dpair = (pair is not None) if need_dpair is None else bool(need_dpair)
+    if need_dmask and mask is None:
+        raise ValueError("dmask requested without a mask")
+    if need_dpair and pair is None:
+        raise ValueError("dpair requested without a pair bias")
+    for name, t, shape, dt in (("k", k, q.shape, q.dtype), ("v", v, q.shape, q.dtype),
+                               ("mask", mask, (B, N, 1, 1, S), q.dtype), ("pair", pair, (B, 1, H, S, S), q.dtype),
+                               ("o", o, q.shape, q.dtype), ("lse", lse, (B, N, H, S), torch.float32),
+                               ("do", do, q.shape, q.dtype)):
+        if t is None:
+            continue
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if t.dtype != dt:
+            raise TypeError(f"{name} dtype {t.dtype}, expected {dt}")
+        if t.device != q.device:
+            raise ValueError(f"{name} is on {t.device}, q on {q.device}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if q.device.type != "cuda":
+        raise ValueError("tensors must be on a CUDA device")
+    need = evo_attn_bwd_workspace_size(B, N, S, H, D)
+    if need < 0:
+        raise EvoAttnError(need, "evo_attn_bwd_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    dmask = torch.empty_like(mask) if need_dmask else None
+    dpair = torch.empty_like(pair) if need_dpair else None
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    status = evo_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(mask), _ptr(pair), o.data_ptr(),
+                          lse.data_ptr(), do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), _ptr(dmask),
+                          _ptr(dpair), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                          B, N, S, H, D, _DTYPES[q.dtype], stream.cuda_stream)
+    if status != EVO_OK:
+        raise EvoAttnError(status, "evo_attn_bwd")
+    return dq, dk, dv, dmask, dpair

@@ -21,6 +21,7 @@
 #include "common.cuh"
 #include "fwd_tri_sm100.cuh"
 #include "fwd_f32.cuh"
+#include "bwd_simt.cuh"
 
 namespace {
 
@@ -544,4 +545,195 @@ extern "C" EVO_API int evo_attn_fwd_host(const void* Qh, const void* Kh, const v
         cudaStreamWaitEvent(cs, hp.done, 0) != cudaSuccess || cudaStreamWaitEvent(cs, hp.in[0], 0) != cudaSuccess)
         return EVO_ERR_CUDA;
     return st;
+}
+
+// ---------------------------------------------------------------- backward
+
+namespace {
+
+// Workspace of evo_attn_bwd: fp32 sections, each starting on a 256-byte
+// boundary, in this order (byte offsets from the workspace pointer).
+struct BwdLayout {
+    int64_t cmask = 0;      // [B * N]        mask rebase c of each (b, n)
+    int64_t lse_r = 0;      // [B, N, H, S]   LSE - c (natural log)
+    int64_t delta = 0;      // [B, N, H, S]   dO . O
+    int64_t dq_acc = 0;     // [B, N, S, H, D] dQ partial sums (tensor-core path)
+    int64_t dmask_acc = 0;  // [B, N, S]      dmask partial sums (tensor-core path)
+    int64_t dpair_acc = 0;  // [B, H, S, S]   dpair partial sums (tensor-core path)
+    int64_t total = 0;
+};
+
+bool bwd_layout(int64_t B, int64_t N, int64_t S, int64_t H, int64_t D, BwdLayout* L) {
+    int64_t bn, bns, bnhs, bnshd, bh, bhs, bhss;
+    if (!mul_ok(B, N, &bn) || !mul_ok(bn, S, &bns) || !mul_ok(bns, H, &bnhs) || !mul_ok(bnhs, D, &bnshd) ||
+        !mul_ok(B, H, &bh) || !mul_ok(bh, S, &bhs) || !mul_ok(bhs, S, &bhss))
+        return false;
+    int64_t off = 0;
+    auto take = [&off](int64_t elems, int64_t* at) {
+        int64_t bytes;
+        if (!mul_ok(elems, 4, &bytes) || bytes > INT64_MAX - off - 256) return false;
+        *at = off;
+        off += (bytes + 255) / 256 * 256;
+        return true;
+    };
+    if (!take(bn, &L->cmask) || !take(bnhs, &L->lse_r) || !take(bnhs, &L->delta) || !take(bnshd, &L->dq_acc) ||
+        !take(bns, &L->dmask_acc) || !take(bhss, &L->dpair_acc))
+        return false;
+    L->total = off;
+    return true;
+}
+
+// Every argument check of evo_attn_bwd that needs no CUDA call, in the order
+// the header lists them.  On success *tensor_core says which path runs.
+int check_bwd(const void* Q, const void* K, const void* V, const void* mask_bias, const void* pair_bias,
+              const void* O, const float* LSE, const void* dO, void* dQ, void* dK, void* dV, void* dmask,
+              void* dpair, void* workspace, int64_t workspace_bytes, int64_t B, int64_t N, int64_t S, int64_t H,
+              int64_t D, int dtype, bool* tensor_core) {
+    *tensor_core = false;
+    if (B < 0 || N < 0 || S < 0 || H < 0 || D < 0 || workspace_bytes < 0) return EVO_ERR_INVALID_ARG;
+    if (dtype != EVO_DTYPE_BF16 && dtype != EVO_DTYPE_FP32 && dtype != EVO_DTYPE_FP16) return EVO_ERR_UNSUPPORTED_DTYPE;
+    if (D == 0 || D > evo::kF32MaxD) return EVO_ERR_UNSUPPORTED_SHAPE;
+    if (B == 0 || N == 0 || S == 0 || H == 0) return EVO_OK;  // nothing to compute
+    if (!Q || !K || !V || !O || !LSE || !dO || !dQ || !dK || !dV || !workspace) return EVO_ERR_INVALID_ARG;
+    if ((dmask && !mask_bias) || (dpair && !pair_bias)) return EVO_ERR_INVALID_ARG;
+
+    const int64_t es = dtype == EVO_DTYPE_FP32 ? 4 : 2;
+    int64_t bn, bns, bnsh, qkv_elems, qkv_bytes, mask_bytes, bh, pair_elems, pair_bytes, lse_bytes;
+    if (!mul_ok(B, N, &bn) || !mul_ok(bn, S, &bns) || !mul_ok(bns, H, &bnsh) || !mul_ok(bnsh, D, &qkv_elems) ||
+        !mul_ok(qkv_elems, es, &qkv_bytes) || !mul_ok(bns, es, &mask_bytes) || !mul_ok(B, H, &bh) ||
+        !mul_ok(bh, S, &pair_elems) || !mul_ok(pair_elems, S, &pair_elems) ||
+        !mul_ok(pair_elems, es, &pair_bytes) || !mul_ok(bnsh, 4, &lse_bytes))
+        return EVO_ERR_UNSUPPORTED_SHAPE;
+    BwdLayout L;
+    if (!bwd_layout(B, N, S, H, D, &L)) return EVO_ERR_UNSUPPORTED_SHAPE;
+    if (workspace_bytes < L.total) return EVO_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return EVO_ERR_MISALIGNED;
+
+    // outputs (and the workspace) must not overlap each other or any input
+    const void* ins[8] = {Q, K, V, mask_bias, pair_bias, O, LSE, dO};
+    const int64_t in_bytes[8] = {qkv_bytes, qkv_bytes, qkv_bytes, mask_bytes, pair_bytes, qkv_bytes, lse_bytes,
+                                 qkv_bytes};
+    const void* outs[6] = {dQ, dK, dV, dmask, dpair, workspace};
+    const int64_t out_bytes[6] = {qkv_bytes, qkv_bytes, qkv_bytes, mask_bytes, pair_bytes, L.total};
+    for (int a = 0; a < 6; ++a) {
+        for (int b = a + 1; b < 6; ++b)
+            if (overlap(outs[a], out_bytes[a], outs[b], out_bytes[b])) return EVO_ERR_INVALID_ARG;
+        for (int i = 0; i < 8; ++i)
+            if (overlap(outs[a], out_bytes[a], ins[i], in_bytes[i])) return EVO_ERR_INVALID_ARG;
+    }
+
+    if (!aligned(LSE, 4)) return EVO_ERR_MISALIGNED;
+    const int64_t int_max = 2147483647;
+    if (S > int_max || N > int_max || H > int_max || bn > int_max) return EVO_ERR_UNSUPPORTED_SHAPE;
+    // the SIMT kernels run one thread per (slice, row, 32 columns), per
+    // (b, n, key) and per pair-bias element, in blocks of 128
+    const int64_t nch = (D + evo::kBwdChunk - 1) / evo::kBwdChunk;
+    int64_t threads;
+    if (!mul_ok(bnsh, nch, &threads) || threads / 128 >= int_max || pair_elems / 128 >= int_max)
+        return EVO_ERR_UNSUPPORTED_SHAPE;
+    for (const void* ptr : {Q, K, V, O, dO, static_cast<const void*>(dQ), static_cast<const void*>(dK),
+                            static_cast<const void*>(dV), mask_bias, pair_bias, static_cast<const void*>(dmask),
+                            static_cast<const void*>(dpair)})
+        if (ptr && !aligned(ptr, uintptr_t(es))) return EVO_ERR_MISALIGNED;
+    return EVO_OK;
+}
+
+template <typename T>
+int launch_bwd_simt(const void* Q, const void* K, const void* V, const void* mask_bias, const void* pair_bias,
+                    const void* O, const float* LSE, const void* dO, void* dQ, void* dK, void* dV, void* dmask,
+                    void* dpair, void* workspace, int64_t B, int64_t N, int64_t S, int64_t H, int64_t D,
+                    cudaStream_t st) {
+    BwdLayout L;
+    bwd_layout(B, N, S, H, D, &L);  // checked by check_bwd
+    char* ws = static_cast<char*>(workspace);
+    evo::BwdParams<T> p;
+    p.q = static_cast<const T*>(Q);
+    p.k = static_cast<const T*>(K);
+    p.v = static_cast<const T*>(V);
+    p.mask = static_cast<const T*>(mask_bias);
+    p.pair = static_cast<const T*>(pair_bias);
+    p.o = static_cast<const T*>(O);
+    p.dout = static_cast<const T*>(dO);
+    p.lse = LSE;
+    p.dq = static_cast<T*>(dQ);
+    p.dk = static_cast<T*>(dK);
+    p.dv = static_cast<T*>(dV);
+    p.dmask = static_cast<T*>(dmask);
+    p.dpair = static_cast<T*>(dpair);
+    p.cmask = reinterpret_cast<float*>(ws + L.cmask);
+    p.lse_r = reinterpret_cast<float*>(ws + L.lse_r);
+    p.delta = reinterpret_cast<float*>(ws + L.delta);
+    p.B = int(B);
+    p.N = int(N);
+    p.S = int(S);
+    p.H = int(H);
+    p.D = int(D);
+    p.scale = float(1.0 / std::sqrt(double(D)));
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = st;
+    cfg.gridDim = dim3(unsigned(B * N), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    if (cudaLaunchKernelEx(&cfg, evo::evo_bwd_rowstats_kernel<T>, p) != cudaSuccess) return EVO_ERR_CUDA;
+    const long long nch = (D + evo::kBwdChunk - 1) / evo::kBwdChunk;
+    const long long rows = (long long)B * N * H * S * nch;
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.gridDim = dim3(unsigned((rows + 127) / 128), 1, 1);
+    if (cudaLaunchKernelEx(&cfg, evo::evo_bwd_simt_kv_kernel<T>, p, rows) != cudaSuccess) return EVO_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, evo::evo_bwd_simt_q_kernel<T>, p, rows) != cudaSuccess) return EVO_ERR_CUDA;
+    if (dmask) {
+        const long long n = (long long)B * N * S;
+        cfg.gridDim = dim3(unsigned((n + 127) / 128), 1, 1);
+        if (cudaLaunchKernelEx(&cfg, evo::evo_bwd_simt_dmask_kernel<T>, p, n) != cudaSuccess) return EVO_ERR_CUDA;
+    }
+    if (dpair) {
+        const long long n = (long long)B * H * S * S;
+        cfg.gridDim = dim3(unsigned((n + 127) / 128), 1, 1);
+        if (cudaLaunchKernelEx(&cfg, evo::evo_bwd_simt_dpair_kernel<T>, p, n) != cudaSuccess) return EVO_ERR_CUDA;
+    }
+    return EVO_OK;
+}
+
+int launch_bwd(int dev, bool tensor_core, const void* Q, const void* K, const void* V, const void* mask_bias,
+               const void* pair_bias, const void* O, const float* LSE, const void* dO, void* dQ, void* dK, void* dV,
+               void* dmask, void* dpair, void* workspace, int64_t B, int64_t N, int64_t S, int64_t H, int64_t D,
+               int dtype, cudaStream_t st) {
+    (void)dev;
+    (void)tensor_core;
+#define EVO_BWD_SIMT(T)                                                                                         \
+    return launch_bwd_simt<T>(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair, workspace, B, \
+                              N, S, H, D, st)
+    if (dtype == EVO_DTYPE_FP32) EVO_BWD_SIMT(float);
+    if (dtype == EVO_DTYPE_FP16) EVO_BWD_SIMT(__half);
+    EVO_BWD_SIMT(uint16_t);
+#undef EVO_BWD_SIMT
+}
+
+}  // namespace
+
+extern "C" EVO_API int64_t evo_attn_bwd_workspace_size(int64_t B, int64_t N, int64_t S, int64_t H, int64_t D) {
+    if (B < 0 || N < 0 || S < 0 || H < 0 || D < 0) return EVO_ERR_INVALID_ARG;
+    BwdLayout L;
+    if (!bwd_layout(B, N, S, H, D, &L)) return EVO_ERR_UNSUPPORTED_SHAPE;
+    return L.total;
+}
+
+extern "C" EVO_API int evo_attn_bwd(const void* Q, const void* K, const void* V, const void* mask_bias,
+                                    const void* pair_bias, const void* O, const float* LSE, const void* dO,
+                                    void* dQ, void* dK, void* dV, void* dmask, void* dpair, void* workspace,
+                                    int64_t workspace_bytes, int64_t B, int64_t N, int64_t S, int64_t H,
+                                    int64_t D, int dtype, evo_stream_t stream) {
+    bool tensor_core = false;
+    const int st = check_bwd(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair, workspace,
+                             workspace_bytes, B, N, S, H, D, dtype, &tensor_core);
+    if (st != EVO_OK || B == 0 || N == 0 || S == 0 || H == 0) return st;
+    RelaxedCapture relaxed;
+    DeviceScope scope;
+    const int dev = select_call_device(Q, K, V, O, LSE, mask_bias, pair_bias, scope);
+    if (dev < 0) return dev;
+    for (const void* ptr : {dO, static_cast<const void*>(dQ), static_cast<const void*>(dK),
+                            static_cast<const void*>(dV), static_cast<const void*>(dmask),
+                            static_cast<const void*>(dpair), static_cast<const void*>(workspace)})
+        if (ptr != nullptr && device_of(ptr) != dev) return EVO_ERR_INVALID_ARG;
+    return launch_bwd(dev, tensor_core, Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair,
+                      workspace, B, N, S, H, D, dtype, reinterpret_cast<cudaStream_t>(stream));
 }
