@@ -218,11 +218,23 @@ EVO_API int64_t evo_attn_bwd_workspace_size(int64_t B, int64_t N, int64_t S, int
  * near -1e9 has lost the digits that matter.  A row with no finite logit
  * (every key -inf) has no weights and contributes zero to every gradient.
  *
- * Supported envelope: every dtype, 1 <= D <= 128, any S, with plain fp32
- * FMA arithmetic (recomputing the weights per gradient); pointers aligned to
- * the element size (LSE to 4 bytes).  The gradients of a call are computed
- * by several kernels on `stream` and are complete once its work there is.
- * Outputs and workspace must not overlap each other or any input.
+ * Supported envelope: every dtype, 1 <= D <= 128, any S; pointers aligned to
+ * the element size (LSE to 4 bytes).  Two implementations:
+ *   - tcgen05 tensor cores for EVO_DTYPE_BF16 / EVO_DTYPE_FP16 with D in
+ *     {16, 32, 64}, no pair bias or S a multiple of 8, and Q, K, V, dO, dQ,
+ *     dK, dV (and the pair bias) 16-byte aligned: S, dP, dV, dK and dQ are
+ *     MMAs with fp32 accumulation; the weights p and logit gradients dt
+ *     enter them rounded to the input type; dQ, dmask and dpair are summed
+ *     in fp32 in the workspace (with atomic adds, so the order of the
+ *     additions, and the last bits of those three gradients, can vary from
+ *     call to call) and rounded at the end;
+ *   - plain fp32 FMA arithmetic for every other accepted call (fp32 inputs,
+ *     other head dims, pair-bias rows that are not 16-byte units, less
+ *     aligned pointers), recomputing the weights per gradient; deterministic,
+ *     and far slower.
+ * The gradients of a call are computed by several kernels (and zeroing
+ * copies) on `stream` and are complete once its work there is.  Outputs and
+ * workspace must not overlap each other or any input.
  *
  * Returns EVO_OK once the work is enqueued, or a negative evo_status_t
  * (EVO_ERR_INVALID_ARG also for a workspace that is too small, or a gradient

@@ -61,15 +61,20 @@ def test_bwd_tiny_fp32():
     compare(case, 0, "tiny_fp32")
 
 
-# (B, N, S, H, D, mask, pair, spike_frac, fully_masked)
+# (B, N, S, H, D, mask, pair, spike_frac, fully_masked).  bf16 with D in
+# {16, 32, 64} and a pair bias whose rows are whole 16-byte units (or none)
+# runs on the tensor-core kernel; the rest on the SIMT kernels.
 BF16_CASES = [
-    (1, 4, 200, 2, 32, "tail", True, 0.01, 1),
-    (1, 3, 130, 2, 64, "head", True, 0.0, 0),
-    (2, 3, 96, 3, 16, "bernoulli", False, 0.0, 0),
-    (1, 2, 77, 2, 48, "tail", True, 0.0, 0),
-    (1, 3, 160, 2, 32, "neg_inf", True, 0.0, 0),
-    (1, 2, 64, 2, 32, "none", True, 0.0, 0),
-    (1, 1, 1, 1, 32, "zero", True, 0.0, 0),
+    (1, 4, 200, 2, 32, "tail", True, 0.01, 1),      # tensor cores, ragged blocks, a fully masked n
+    (1, 3, 136, 2, 64, "head", True, 0.0, 0),       # tensor cores, D = 64
+    (2, 3, 96, 3, 16, "bernoulli", False, 0.0, 0),  # tensor cores, D = 16, no pair bias
+    (1, 2, 256, 2, 16, "tail", True, 0.01, 0),      # tensor cores, D = 16, two whole blocks
+    (1, 3, 160, 2, 32, "neg_inf", True, 0.0, 0),    # tensor cores, -inf mask entries
+    (1, 2, 64, 2, 32, "none", True, 0.0, 0),        # tensor cores, no mask
+    (1, 2, 384, 4, 32, "tail", False, 0.0, 1),      # tensor cores, no pair bias, several blocks
+    (1, 3, 130, 2, 64, "head", True, 0.0, 0),       # SIMT: pair rows not 16-byte units
+    (1, 2, 77, 2, 48, "tail", True, 0.0, 0),        # SIMT: head dim 48
+    (1, 1, 1, 1, 32, "zero", True, 0.0, 0),         # SIMT: S = 1
 ]
 
 
@@ -84,6 +89,13 @@ def test_bwd_bf16(shape):
 def test_bwd_fp32_random():
     case = W.random_case(2, 3, 77, 2, 24, torch.float32, seed=5, mask="tail", pair=True, fully_masked=1)
     compare(case, 5, "fp32 random")
+
+
+def test_bwd_fp16_tensor_cores():
+    case = W.random_case(1, 3, 264, 2, 64, torch.float16, seed=9, mask="bernoulli", pair=True, spike_frac=0.01)
+    compare(case, 9, "fp16 D=64 tensor cores")
+    case = W.random_case(2, 2, 128, 2, 32, torch.float16, seed=10, mask="none", pair=False)
+    compare(case, 10, "fp16 D=32 tensor cores, no biases")
 
 
 def test_bwd_fp16_fully_masked_rows_are_empty():

@@ -12,7 +12,9 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
+#include <type_traits>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -22,6 +24,7 @@
 #include "fwd_tri_sm100.cuh"
 #include "fwd_f32.cuh"
 #include "bwd_simt.cuh"
+#include "bwd_tri_sm100.cuh"
 
 namespace {
 
@@ -635,14 +638,22 @@ int check_bwd(const void* Q, const void* K, const void* V, const void* mask_bias
                             static_cast<const void*>(dV), mask_bias, pair_bias, static_cast<const void*>(dmask),
                             static_cast<const void*>(dpair)})
         if (ptr && !aligned(ptr, uintptr_t(es))) return EVO_ERR_MISALIGNED;
+    // the tensor-core path: 16-bit types, D in {16, 32, 64}, pair-bias rows in
+    // whole 16-byte units (loaded by TMA), the tiles 16-byte aligned; every
+    // other accepted call runs on the SIMT kernels
+    int64_t units;
+    *tensor_core = dtype != EVO_DTYPE_FP32 && (D == 16 || D == 32 || D == 64) &&
+                   (pair_bias == nullptr || (S % 8 == 0 && aligned(pair_bias, 16))) && aligned(Q, 16) &&
+                   aligned(K, 16) && aligned(V, 16) && aligned(dO, 16) && aligned(dQ, 16) && aligned(dK, 16) &&
+                   aligned(dV, 16) && mul_ok(bnsh / S, (S + evo::kBN - 1) / evo::kBN, &units) && units <= int_max;
     return EVO_OK;
 }
 
 template <typename T>
-int launch_bwd_simt(const void* Q, const void* K, const void* V, const void* mask_bias, const void* pair_bias,
-                    const void* O, const float* LSE, const void* dO, void* dQ, void* dK, void* dV, void* dmask,
-                    void* dpair, void* workspace, int64_t B, int64_t N, int64_t S, int64_t H, int64_t D,
-                    cudaStream_t st) {
+evo::BwdParams<T> make_bwd_params(const void* Q, const void* K, const void* V, const void* mask_bias,
+                                  const void* pair_bias, const void* O, const float* LSE, const void* dO, void* dQ,
+                                  void* dK, void* dV, void* dmask, void* dpair, void* workspace, int64_t B,
+                                  int64_t N, int64_t S, int64_t H, int64_t D) {
     BwdLayout L;
     bwd_layout(B, N, S, H, D, &L);  // checked by check_bwd
     char* ws = static_cast<char*>(workspace);
@@ -669,11 +680,29 @@ int launch_bwd_simt(const void* Q, const void* K, const void* V, const void* mas
     p.H = int(H);
     p.D = int(D);
     p.scale = float(1.0 / std::sqrt(double(D)));
+    return p;
+}
+
+// delta, the rebased LSE and the mask shift of every row (both paths)
+template <typename T>
+int launch_rowstats(const evo::BwdParams<T>& p, int64_t B, int64_t N, cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
     cfg.stream = st;
     cfg.gridDim = dim3(unsigned(B * N), 1, 1);
     cfg.blockDim = dim3(256, 1, 1);
-    if (cudaLaunchKernelEx(&cfg, evo::evo_bwd_rowstats_kernel<T>, p) != cudaSuccess) return EVO_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, evo::evo_bwd_rowstats_kernel<T>, p) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+}
+
+template <typename T>
+int launch_bwd_simt(const void* Q, const void* K, const void* V, const void* mask_bias, const void* pair_bias,
+                    const void* O, const float* LSE, const void* dO, void* dQ, void* dK, void* dV, void* dmask,
+                    void* dpair, void* workspace, int64_t B, int64_t N, int64_t S, int64_t H, int64_t D,
+                    cudaStream_t st) {
+    const evo::BwdParams<T> p = make_bwd_params<T>(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask,
+                                                   dpair, workspace, B, N, S, H, D);
+    if (launch_rowstats<T>(p, B, N, st) != EVO_OK) return EVO_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = st;
     const long long nch = (D + evo::kBwdChunk - 1) / evo::kBwdChunk;
     const long long rows = (long long)B * N * H * S * nch;
     cfg.blockDim = dim3(128, 1, 1);
@@ -693,12 +722,103 @@ int launch_bwd_simt(const void* Q, const void* K, const void* V, const void* mas
     return EVO_OK;
 }
 
+// The tcgen05 backward: fp32 accumulators zeroed, row statistics, the
+// persistent gradient kernel, then the rounding of the fp32 sums.
+template <int D, bool HAS_PAIR, bool F16>
+int launch_bwd_tri(int dev, const void* Q, const void* K, const void* V, const void* mask_bias,
+                   const void* pair_bias, const void* O, const float* LSE, const void* dO, void* dQ, void* dK,
+                   void* dV, void* dmask, void* dpair, void* workspace, int64_t B, int64_t N, int64_t S, int64_t H,
+                   cudaStream_t st) {
+    using C = evo::BwdCfg<D, HAS_PAIR, F16>;
+    using T = typename std::conditional<F16, __half, uint16_t>::type;
+    auto kernel = evo::evo_bwd_tri_kernel<D, HAS_PAIR, F16>;
+    static AttrOnce attr;
+    if (!attr.ensure(dev, kernel, C::SMEM_BYTES)) return EVO_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return EVO_ERR_CUDA;
+    const CUtensorMapDataType dt = F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUtensorMap tq, tk, tv, tdo, tp;
+    std::memset(&tp, 0, sizeof(tp));
+    if (!encode_qkv(&tq, Q, B * N, S, H, D, 16, dt) || !encode_qkv(&tk, K, B * N, S, H, D, 16, dt) ||
+        !encode_qkv(&tv, V, B * N, S, H, D, 16, dt) || !encode_qkv(&tdo, dO, B * N, S, H, D, 16, dt))
+        return EVO_ERR_CUDA;
+    if (HAS_PAIR && !encode_pair(&tp, pair_bias, B * H, S, dt)) return EVO_ERR_CUDA;
+
+    BwdLayout L;
+    bwd_layout(B, N, S, H, D, &L);
+    char* ws = static_cast<char*>(workspace);
+    const long long n_q = (long long)B * N * S * H * D, n_m = (long long)B * N * S, n_p = (long long)B * H * S * S;
+    if (cudaMemsetAsync(ws + L.dq_acc, 0, size_t(n_q) * 4, st) != cudaSuccess ||
+        (dmask && cudaMemsetAsync(ws + L.dmask_acc, 0, size_t(n_m) * 4, st) != cudaSuccess) ||
+        (dpair && cudaMemsetAsync(ws + L.dpair_acc, 0, size_t(n_p) * 4, st) != cudaSuccess))
+        return EVO_ERR_CUDA;
+    const evo::BwdParams<T> bp = make_bwd_params<T>(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask,
+                                                    dpair, workspace, B, N, S, H, D);
+    if (launch_rowstats<T>(bp, B, N, st) != EVO_OK) return EVO_ERR_CUDA;
+
+    evo::BwdTriParams p;
+    p.mask = static_cast<const uint16_t*>(mask_bias);
+    p.cmask = bp.cmask;
+    p.lse_r = bp.lse_r;
+    p.delta = bp.delta;
+    p.dk = static_cast<uint16_t*>(dK);
+    p.dv = static_cast<uint16_t*>(dV);
+    p.dq_acc = reinterpret_cast<float*>(ws + L.dq_acc);
+    p.dmask_acc = dmask ? reinterpret_cast<float*>(ws + L.dmask_acc) : nullptr;
+    p.dpair_acc = dpair ? reinterpret_cast<float*>(ws + L.dpair_acc) : nullptr;
+    p.N = int(N);
+    p.S = int(S);
+    p.H = int(H);
+    p.num_kb = int((S + evo::kBN - 1) / evo::kBN);
+    p.num_qb = int((S + evo::kBM - 1) / evo::kBM);
+    p.num_units = int(B * N * H * p.num_kb);
+    p.scale = float(1.0 / std::sqrt(double(D)));
+    p.scale_log2 = float(1.4426950408889634 / std::sqrt(double(D)));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(p.num_units < sms ? p.num_units : sms), 1, 1);
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = st;
+    if (cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, tdo, tp, p) != cudaSuccess) return EVO_ERR_CUDA;
+
+    cudaLaunchConfig_t pc = {};
+    const long long work = std::max(n_q / 4, std::max(dmask ? n_m : 0ll, dpair ? n_p : 0ll));
+    pc.gridDim = dim3(unsigned(std::min<long long>((work + 255) / 256, (long long)sms * 16)), 1, 1);
+    pc.blockDim = dim3(256, 1, 1);
+    pc.stream = st;
+    return cudaLaunchKernelEx(&pc, evo::evo_bwd_post_kernel<F16>, (const float*)p.dq_acc, static_cast<uint16_t*>(dQ),
+                              n_q, p.scale, (const float*)p.dmask_acc, static_cast<uint16_t*>(dmask), n_m,
+                              (const float*)p.dpair_acc, static_cast<uint16_t*>(dpair), n_p) == cudaSuccess
+               ? EVO_OK
+               : EVO_ERR_CUDA;
+}
+
 int launch_bwd(int dev, bool tensor_core, const void* Q, const void* K, const void* V, const void* mask_bias,
                const void* pair_bias, const void* O, const float* LSE, const void* dO, void* dQ, void* dK, void* dV,
                void* dmask, void* dpair, void* workspace, int64_t B, int64_t N, int64_t S, int64_t H, int64_t D,
                int dtype, cudaStream_t st) {
-    (void)dev;
-    (void)tensor_core;
+    if (tensor_core) {
+        if (encode_fn() == nullptr) return EVO_ERR_CUDA;
+        const bool has_pair = pair_bias != nullptr, f16 = dtype == EVO_DTYPE_FP16;
+#define EVO_BWD_TRI(DD, PAIR, F)                                                                              \
+    return launch_bwd_tri<DD, PAIR, F>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair, \
+                                       workspace, B, N, S, H, st)
+#define EVO_BWD_TRI_D(DD)                                 \
+    if (f16) {                                            \
+        if (has_pair) EVO_BWD_TRI(DD, true, true);        \
+        EVO_BWD_TRI(DD, false, true);                     \
+    }                                                     \
+    if (has_pair) EVO_BWD_TRI(DD, true, false);           \
+    EVO_BWD_TRI(DD, false, false)
+        switch (D) {
+            case 16: EVO_BWD_TRI_D(16);
+            case 32: EVO_BWD_TRI_D(32);
+            default: EVO_BWD_TRI_D(64);
+        }
+#undef EVO_BWD_TRI_D
+#undef EVO_BWD_TRI
+    }
 #define EVO_BWD_SIMT(T)                                                                                         \
     return launch_bwd_simt<T>(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair, workspace, B, \
                               N, S, H, D, st)
