@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="tri_1024", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
+                    help="fwd: the forward pass (the headline metric); bwd: the backward pass "
+                         "(evo_attn_bwd: dQ, dK, dV and the requested bias gradients)")
     ap.add_argument("--e2e-steps", type=int, default=5,
                     help="steps of the host-memory leg (0 skips it; e2e is then null)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -427,12 +430,119 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def bwd_flops(wl) -> int:
+    # five products of 2*S*S*D each per (b, n, h): S = Q K^T (recomputed),
+    # dP = dO V^T, dV = P^T dO, dK = dT^T Q, dQ = dT K
+    return 10 * wl.B * wl.N * wl.H * wl.S * wl.S * wl.D
+
+
+def upstream_grad(case, seed: int):
+    import numpy as np
+    rng = np.random.Generator(np.random.PCG64(50_000 + seed))
+    return torch.from_numpy(rng.standard_normal(case.q.shape, dtype=np.float32)).to(case.q.dtype)
+
+
+def cpu_baseline_bwd(case, do, args, target_s: float = 10.0):
+    """The oracle's backward on random (b, n, h) slices until about
+    `target_s` seconds have been spent."""
+    import oracle
+    B, N, S, H, D = case.shape
+    cores = oracle.max_threads()
+    rng = torch.Generator().manual_seed(args.seed)
+    done_sec = 0.0
+    n_slices = 0
+    while done_sec < target_s and n_slices < B * N * H:
+        idx = torch.randint(0, B * N * H, (cores,), generator=rng).tolist()
+        sl = [(i // (N * H), (i // H) % N, i % H) for i in idx]
+        t0 = time.perf_counter()
+        oracle.default().attention_bwd_slices(case.q, case.k, case.v, case.mask, case.pair, do, sl)
+        done_sec += time.perf_counter() - t0
+        n_slices += len(sl)
+    flops = 10.0 * S * S * D * n_slices
+    return {"value": flops / done_sec / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "cpu": cpu_model(), "nproc": os.cpu_count(),
+            "sample": f"backward of {n_slices} random (b,n,h) slices of {args.workload} "
+                      f"({flops / 1e9:.0f} GFLOP in {done_sec:.1f} s, float64 C, OpenMP)"}
+
+
+def run_ours_bwd(args, rank, world, local):
+    """The backward pass: each step is one evo_attn_bwd call (zeroing of the
+    fp32 accumulators, row statistics, the gradient kernel, the rounding
+    kernel) on the forward's outputs, every gradient requested."""
+    import triangle_biased_attention_b200 as evo
+    wl = W.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    case = W.make_case(args.workload, args.seed + rank)
+    do_h = upstream_grad(case, args.seed + rank)
+    q, k, v, do = (t.to(dev) for t in (case.q, case.k, case.v, do_h))
+    mask = case.mask.to(dev) if case.mask is not None else None
+    pair = case.pair.to(dev) if case.pair is not None else None
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        o, lse = evo.evo_attn(q, k, v, mask, pair, stream=stream)
+    B, N, S, H, D = q.shape
+    ws = torch.empty(evo.evo_attn_bwd_workspace_size(B, N, S, H, D), dtype=torch.uint8, device=dev)
+
+    def step():
+        return evo.evo_attn_backward(q, k, v, mask, pair, o, lse, do, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    status = evo.evo_attn_sync_status(stream.cuda_stream)
+    if status != evo.EVO_OK:
+        raise RuntimeError(f"kernel status {status}: {evo.evo_attn_strerror(status)}")
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with sampler:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(args.steps):
+                step()
+            stop.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = start.elapsed_time(stop)
+    status = evo.evo_attn_sync_status(stream.cuda_stream)
+    if status != evo.EVO_OK:
+        raise RuntimeError(f"kernel status {status}: {evo.evo_attn_strerror(status)}")
+    ms_max = max_over_ranks(ms, world, dev)
+    flops = bwd_flops(wl)
+    value = world * flops * args.steps / (ms_max * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms / args.steps * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst figure)" if peak_src == "measured"
+            else "fallback (6.65 TB/s, 1.59 PFLOP/s)",
+            "alg_flops_per_launch": flops,
+            "timed": "whole evo_attn_bwd call (3 kernels and the zeroing copies of the fp32 sums)"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_bwd(case, do_h, args)
+    if rank == 0:
+        line = {
+            "metric": "Evoformer attn bwd TFLOP/s (dQ, dK, dV, dmask, dpair; 10*B*N*H*S^2*D flops)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded numpy PCG64, bf16)",
+            "config": workload_config(wl), "roofline": roof, "cpu_baseline": cpu, "e2e": None,
+            "gpu_launches": 3 * args.steps, "kernel": "evo_bwd_tri_kernel", "clocks": sampler.record(),
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     rank, world, local = dist_setup(args)
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.which == "bwd":
+            run_ours_bwd(args, rank, world, local)
         else:
             run_ours(args, rank, world, local)
     finally:

@@ -193,7 +193,7 @@ def test_bwd_workspace_size(lib):
     size = evo.evo_attn_bwd_workspace_size(B, N, S, H, D)
     r = lambda b: (b + 255) // 256 * 256
     expect = (r(4 * B * N) + 2 * r(4 * B * N * H * S) + r(4 * B * N * S * H * D) + r(4 * B * N * S)
-              + r(4 * B * H * S * S))
+              + r(4 * B * H * S * S) + r(4 * (B * N + 1)))
     assert size == expect
     assert evo.evo_attn_bwd_workspace_size(-1, N, S, H, D) == evo.EVO_ERR_INVALID_ARG
     assert evo.evo_attn_bwd_workspace_size(1 << 40, 1 << 40, S, H, D) == evo.EVO_ERR_UNSUPPORTED_SHAPE

@@ -129,3 +129,31 @@ def test_bwd_rejects_overlapping_outputs_on_device():
     assert evo.evo_attn_bwd(*args(dk.data_ptr())) == evo.EVO_ERR_INVALID_ARG    # dQ over dK
     assert evo.evo_attn_bwd(*args(dq.data_ptr())) == evo.EVO_OK
     assert evo.evo_attn_sync_status() == evo.EVO_OK
+
+
+def test_bwd_tri_1024_sampled():
+    """The backward at the full triangle-attention size (B=1, N=S=1024, H=4,
+    D=32, the forward's workload), compared on sampled outputs: dQ, dK, dV of
+    whole (b, n, h) slices, dmask of whole n (all heads), and rows of dpair
+    (each a sum over all 1024 n)."""
+    case = W.make_case("tri_1024", 0)
+    do = _upstream(case, 0)
+    got = run_bwd(case, do)
+    orc = oracle.default()
+    B, N, S, H, D = case.shape
+    fm = case.meta.get("tail", 0)
+    slices = [(0, 0, 0), (0, 517, 3), (0, 1023, 1), (0, 301, 2)]
+    dq, dk, dv, cs = orc.attention_bwd_slices(case.q, case.k, case.v, case.mask, case.pair, do, slices)
+    pick = lambda g: np.stack([g[b, n, :, h, :].double().numpy() for (b, n, h) in slices])
+    check_grads({"dq": pick(got["dq"]), "dk": pick(got["dk"]), "dv": pick(got["dv"])},
+                {"dq": dq, "dk": dk, "dv": dv}, case.dtype, "tri_1024 sampled slices")
+    # dmask of n = 517: the column sums of all four heads' slices
+    hs = [(0, 517, h) for h in range(H)]
+    _, _, _, cs = orc.attention_bwd_slices(case.q, case.k, case.v, case.mask, case.pair, do, hs)
+    ref_m = cs.sum(axis=0)
+    check_grads({"dmask": got["dmask"][0, 517, 0, 0].double().numpy()}, {"dmask": ref_m}, case.dtype,
+                f"tri_1024 dmask (tail {fm})")
+    rows = [(0, 0, 5), (0, 2, 700), (0, 3, 1023)]
+    ref_p = orc.pair_grad_rows(case.q, case.k, case.v, case.mask, case.pair, do, rows, chunk=128)
+    got_p = np.stack([got["dpair"][b, 0, h, i].double().numpy() for (b, h, i) in rows])
+    check_grads({"dpair": got_p}, {"dpair": ref_p}, case.dtype, "tri_1024 dpair rows")

@@ -1,5 +1,5 @@
 // Backward pass of biased attention with plain FMA arithmetic in fp32: the
-// row-statistics kernel that every backward path runs first, and the SIMT
+// row-statistics kernels that every backward path runs first, and the SIMT
 // gradient kernels used for fp32 inputs and for the head dimensions the
 // tensor-core backward does not take.
 //
@@ -23,7 +23,7 @@
 // no weight), so logits and LSE_i - c stay small numbers.  The forward's LSE
 // is an fp32 number; where |c| is large (a row whose every key carries the
 // guide's -1e9) its fp32 rounding (64 at 1e9) would swamp LSE_i - c, so the
-// row statistics kernel recomputes log sum_j exp(t_ij - c) for those rows
+// row statistics recompute log sum_j exp(t_ij - c) for those rows
 // from Q, K and the biases instead of subtracting.
 #pragma once
 
@@ -61,70 +61,139 @@ struct BwdParams {
     float* cmask;   // workspace [B * N]: the mask rebase c of each (b, n)
     float* lse_r;   // workspace [B, N, H, S]: LSE - c (natural log); +inf for rows without a finite logit
     float* delta;   // workspace [B, N, H, S]: dO . O
+    int* shifted;   // workspace [1 + B * N]: count, then the (b, n) whose rows need the LSE recomputed
     int B, N, S, H, D;
+    int vec16;      // 16-bit elements, D % 8 == 0 and O, dO, K 16-byte aligned: rows read 16 bytes at a time
     float scale;    // 1 / sqrt(D)
 };
 
-// One CTA per (b, n): the mask rebase c, then delta and LSE - c of every
-// (h, i) row of that n, one warp per row.
+// The mask rebase c of each (b, n): one warp per (b, n).
 template <typename T>
-__global__ void __launch_bounds__(256) evo_bwd_rowstats_kernel(const BwdParams<T> p) {
-    __shared__ float red[8];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long bn = blockIdx.x;
-    const long long b = bn / p.N;
-    const T* mrow = p.mask ? p.mask + size_t(bn) * p.S : nullptr;
+__global__ void __launch_bounds__(256) evo_bwd_shift_kernel(const BwdParams<T> p, long long bns) {
+    const long long bn = blockIdx.x * 8ll + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (bn >= bns) return;
     float c = 0.f;
-    if (mrow) {
+    if (p.mask != nullptr) {
+        const T* mrow = p.mask + size_t(bn) * p.S;
         float mx = -INFINITY;
-        for (int j = threadIdx.x; j < p.S; j += blockDim.x) mx = fmaxf(mx, ld_elem(mrow, j));
+        for (int j = lane; j < p.S; j += 32) mx = fmaxf(mx, ld_elem(mrow, j));
         mx = warp_max(mx);
-        if (lane == 0) red[warp] = mx;
-        __syncthreads();
-        mx = red[0];
-        for (int w = 1; w < 8; ++w) mx = fmaxf(mx, red[w]);
         c = (mx == -INFINITY) ? 0.f : mx;
     }
-    if (threadIdx.x == 0) p.cmask[bn] = c;
-    const bool recompute = fabsf(c) > kBwdRecomputeAbove;
+    if (lane == 0) {
+        p.cmask[bn] = c;
+        if (fabsf(c) > kBwdRecomputeAbove) p.shifted[1 + atomicAdd(p.shifted, 1)] = int(bn);
+    }
+}
+
+// delta and LSE - c of every row: one thread per (b, n, i, h) row, in memory
+// order (the thread's O and dO rows are D consecutive elements).  Rows of an
+// n whose shift |c| exceeds kBwdRecomputeAbove get their LSE - c from
+// evo_bwd_lse_recompute_kernel instead.
+template <typename T>
+__global__ void __launch_bounds__(256) evo_bwd_rowstats_kernel(const BwdParams<T> p, long long rows) {
+    const long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    if (r >= rows) return;
     const int D = p.D;
-    const size_t row_stride = size_t(p.H) * D;
-    for (int r = warp; r < p.H * p.S; r += 8) {
-        const int h = r / p.S, i = r - h * p.S;
-        const size_t qoff = (size_t(bn) * p.S + i) * row_stride + size_t(h) * D;
-        float acc = 0.f;
-        for (int d = lane; d < D; d += 32) acc = fmaf(ld_elem(p.o, qoff + d), ld_elem(p.dout, qoff + d), acc);
-        acc = warp_sum(acc);
-        const size_t ri = (size_t(bn) * p.H + h) * p.S + i;
-        float lr;
-        if (!recompute) {
-            const float L = p.lse[ri];
-            lr = (L == -INFINITY) ? INFINITY : L - c;
-        } else {
-            // log sum_j exp(t_ij - c) from the inputs
-            const T* prow = p.pair ? p.pair + ((size_t(b) * p.H + h) * p.S + i) * size_t(p.S) : nullptr;
-            float m = -INFINITY, s = 0.f;
-            for (int j = lane; j < p.S; j += 32) {
-                const size_t koff = (size_t(bn) * p.S + j) * row_stride + size_t(h) * D;
-                float dot = 0.f;
-                for (int d = 0; d < D; ++d) dot = fmaf(ld_elem(p.q, qoff + d), ld_elem(p.k, koff + d), dot);
-                float t = dot * p.scale + (ld_elem(mrow, j) - c);
-                if (prow) t += ld_elem(prow, j);
-                if (t > m) {
-                    s = s * expf(m - t) + 1.f;  // m = -inf gives s * 0 + 1
-                    m = t;
-                } else if (t > -INFINITY) {
-                    s += expf(t - m);
+    const int h = int(r % p.H);
+    const long long bi = r / p.H;  // bn * S + i
+    const int i = int(bi % p.S);
+    const long long bn = bi / p.S;
+    const size_t off = size_t(r) * D;
+    float acc = 0.f;
+    bool done = false;
+    if constexpr (sizeof(T) == 2) {
+        if (p.vec16) {
+            // 8 elements per 16-byte load
+            const uint4* o4 = reinterpret_cast<const uint4*>(p.o + off);
+            const uint4* g4 = reinterpret_cast<const uint4*>(p.dout + off);
+            for (int d = 0; d < D / 8; ++d) {
+                const uint4 a = o4[d], g = g4[d];
+                const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const T* ae = reinterpret_cast<const T*>(&aw[e]);
+                    const T* ge = reinterpret_cast<const T*>(&gw[e]);
+                    acc = fmaf(ld_elem(ae, 0), ld_elem(ge, 0), acc);
+                    acc = fmaf(ld_elem(ae, 1), ld_elem(ge, 1), acc);
                 }
             }
-            const float mw = warp_max(m);
-            const float sw = warp_sum(m == -INFINITY ? 0.f : s * expf(m - mw));
-            lr = (mw == -INFINITY) ? INFINITY : mw + logf(sw);
+            done = true;
         }
-        if (lane == 0) {
-            p.delta[ri] = acc;
-            p.lse_r[ri] = lr;
+    }
+    if (!done)
+        for (int d = 0; d < D; ++d) acc = fmaf(ld_elem(p.o, off + d), ld_elem(p.dout, off + d), acc);
+    const size_t ri = (size_t(bn) * p.H + h) * p.S + i;
+    p.delta[ri] = acc;
+    const float c = p.cmask[bn];
+    if (!(fabsf(c) > kBwdRecomputeAbove)) {
+        const float L = p.lse[ri];
+        p.lse_r[ri] = (L == -INFINITY) ? INFINITY : L - c;
+    }
+}
+
+// LSE - c recomputed from the inputs, log sum_j exp(t_ij - c), for the rows
+// of every n whose shift |c| exceeds kBwdRecomputeAbove (the forward's fp32
+// LSE near such a c has lost the digits that matter).  Those n are listed by
+// evo_bwd_shift_kernel; a grid of a few blocks per SM walks their rows, one
+// warp per row, lanes over keys, the query row staged in shared memory.
+template <typename T>
+__global__ void __launch_bounds__(256) evo_bwd_lse_recompute_kernel(const BwdParams<T> p) {
+    __shared__ float qs[8][kF32MaxD];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long rows_per_n = (long long)p.H * p.S;
+    const long long total = (long long)p.shifted[0] * rows_per_n;
+    const long long nwarps = (long long)gridDim.x * 8;
+    const int D = p.D;
+    const size_t row_stride = size_t(p.H) * D;
+    for (long long w = blockIdx.x * 8ll + warp; w < total; w += nwarps) {
+        const long long bn = p.shifted[1 + w / rows_per_n];
+        const int r = int(w % rows_per_n);
+        const int h = r / p.S, i = r - h * p.S;
+        const long long b = bn / p.N;
+        const float c = p.cmask[bn];
+        const T* mrow = p.mask + size_t(bn) * p.S;
+        const size_t qoff = (size_t(bn) * p.S + i) * row_stride + size_t(h) * D;
+        for (int d = lane; d < D; d += 32) qs[warp][d] = ld_elem(p.q, qoff + d);
+        __syncwarp();
+        const T* prow = p.pair ? p.pair + ((size_t(b) * p.H + h) * p.S + i) * size_t(p.S) : nullptr;
+        float m = -INFINITY, s = 0.f;
+        for (int j = lane; j < p.S; j += 32) {
+            const size_t koff = (size_t(bn) * p.S + j) * row_stride + size_t(h) * D;
+            float dot = 0.f;
+            bool done = false;
+            if constexpr (sizeof(T) == 2) {
+                if (p.vec16) {
+                    const uint4* k4 = reinterpret_cast<const uint4*>(p.k + koff);
+                    for (int d8 = 0; d8 < D / 8; ++d8) {
+                        const uint4 kv = __ldg(k4 + d8);
+                        const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const T* ke = reinterpret_cast<const T*>(&kw[e]);
+                            dot = fmaf(qs[warp][8 * d8 + 2 * e], ld_elem(ke, 0), dot);
+                            dot = fmaf(qs[warp][8 * d8 + 2 * e + 1], ld_elem(ke, 1), dot);
+                        }
+                    }
+                    done = true;
+                }
+            }
+            if (!done)
+                for (int d = 0; d < D; ++d) dot = fmaf(qs[warp][d], ld_elem(p.k, koff + d), dot);
+            float t = dot * p.scale + (ld_elem(mrow, j) - c);
+            if (prow) t += ld_elem(prow, j);
+            if (t > m) {
+                s = s * expf(m - t) + 1.f;  // m = -inf gives s * 0 + 1
+                m = t;
+            } else if (t > -INFINITY) {
+                s += expf(t - m);
+            }
         }
+        const float mw = warp_max(m);
+        const float sw = warp_sum(m == -INFINITY ? 0.f : s * expf(m - mw));
+        if (lane == 0) p.lse_r[(size_t(bn) * p.H + h) * p.S + i] = (mw == -INFINITY) ? INFINITY : mw + logf(sw);
+        __syncwarp();
     }
 }
 

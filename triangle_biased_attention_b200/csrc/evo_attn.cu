@@ -563,6 +563,7 @@ struct BwdLayout {
     int64_t dq_acc = 0;     // [B, N, S, H, D] dQ partial sums (tensor-core path)
     int64_t dmask_acc = 0;  // [B, N, S]      dmask partial sums (tensor-core path)
     int64_t dpair_acc = 0;  // [B, H, S, S]   dpair partial sums (tensor-core path)
+    int64_t shifted = 0;    // [1 + B * N] int32: count and list of the (b, n) whose LSE is recomputed
     int64_t total = 0;
 };
 
@@ -580,7 +581,7 @@ bool bwd_layout(int64_t B, int64_t N, int64_t S, int64_t H, int64_t D, BwdLayout
         return true;
     };
     if (!take(bn, &L->cmask) || !take(bnhs, &L->lse_r) || !take(bnhs, &L->delta) || !take(bnshd, &L->dq_acc) ||
-        !take(bns, &L->dmask_acc) || !take(bhss, &L->dpair_acc))
+        !take(bns, &L->dmask_acc) || !take(bhss, &L->dpair_acc) || !take(bn + 1, &L->shifted))
         return false;
     L->total = off;
     return true;
@@ -674,33 +675,48 @@ evo::BwdParams<T> make_bwd_params(const void* Q, const void* K, const void* V, c
     p.cmask = reinterpret_cast<float*>(ws + L.cmask);
     p.lse_r = reinterpret_cast<float*>(ws + L.lse_r);
     p.delta = reinterpret_cast<float*>(ws + L.delta);
+    p.shifted = reinterpret_cast<int*>(ws + L.shifted);
     p.B = int(B);
     p.N = int(N);
     p.S = int(S);
     p.H = int(H);
     p.D = int(D);
     p.scale = float(1.0 / std::sqrt(double(D)));
+    p.vec16 = (sizeof(T) == 2 && D % 8 == 0 && aligned(O, 16) && aligned(dO, 16) && aligned(K, 16)) ? 1 : 0;
     return p;
 }
 
-// delta, the rebased LSE and the mask shift of every row (both paths)
+// The mask shift of every (b, n), then delta and the rebased LSE of every
+// row (recomputed for the rows of a heavily shifted n): both paths.
 template <typename T>
-int launch_rowstats(const evo::BwdParams<T>& p, int64_t B, int64_t N, cudaStream_t st) {
+int launch_rowstats(int dev, const evo::BwdParams<T>& p, int64_t B, int64_t N, int64_t S, int64_t H,
+                    cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
     cfg.stream = st;
-    cfg.gridDim = dim3(unsigned(B * N), 1, 1);
     cfg.blockDim = dim3(256, 1, 1);
-    return cudaLaunchKernelEx(&cfg, evo::evo_bwd_rowstats_kernel<T>, p) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
+    const long long bns = (long long)B * N;
+    if (cudaMemsetAsync(p.shifted, 0, sizeof(int), st) != cudaSuccess) return EVO_ERR_CUDA;
+    cfg.gridDim = dim3(unsigned((bns + 7) / 8), 1, 1);
+    if (cudaLaunchKernelEx(&cfg, evo::evo_bwd_shift_kernel<T>, p, bns) != cudaSuccess) return EVO_ERR_CUDA;
+    const long long rows = bns * S * H;
+    cfg.gridDim = dim3(unsigned((rows + 255) / 256), 1, 1);
+    if (cudaLaunchKernelEx(&cfg, evo::evo_bwd_rowstats_kernel<T>, p, rows) != cudaSuccess) return EVO_ERR_CUDA;
+    if (p.mask == nullptr) return EVO_OK;  // no shift, nothing to recompute
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return EVO_ERR_CUDA;
+    cfg.gridDim = dim3(unsigned(4 * sms), 1, 1);
+    return cudaLaunchKernelEx(&cfg, evo::evo_bwd_lse_recompute_kernel<T>, p) == cudaSuccess ? EVO_OK : EVO_ERR_CUDA;
 }
 
 template <typename T>
-int launch_bwd_simt(const void* Q, const void* K, const void* V, const void* mask_bias, const void* pair_bias,
+int launch_bwd_simt(int dev, const void* Q, const void* K, const void* V, const void* mask_bias, const void* pair_bias,
                     const void* O, const float* LSE, const void* dO, void* dQ, void* dK, void* dV, void* dmask,
                     void* dpair, void* workspace, int64_t B, int64_t N, int64_t S, int64_t H, int64_t D,
                     cudaStream_t st) {
     const evo::BwdParams<T> p = make_bwd_params<T>(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask,
                                                    dpair, workspace, B, N, S, H, D);
-    if (launch_rowstats<T>(p, B, N, st) != EVO_OK) return EVO_ERR_CUDA;
+    if (launch_rowstats<T>(dev, p, B, N, S, H, st) != EVO_OK) return EVO_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.stream = st;
     const long long nch = (D + evo::kBwdChunk - 1) / evo::kBwdChunk;
@@ -755,7 +771,7 @@ int launch_bwd_tri(int dev, const void* Q, const void* K, const void* V, const v
         return EVO_ERR_CUDA;
     const evo::BwdParams<T> bp = make_bwd_params<T>(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask,
                                                     dpair, workspace, B, N, S, H, D);
-    if (launch_rowstats<T>(bp, B, N, st) != EVO_OK) return EVO_ERR_CUDA;
+    if (launch_rowstats<T>(dev, bp, B, N, S, H, st) != EVO_OK) return EVO_ERR_CUDA;
 
     evo::BwdTriParams p;
     p.mask = static_cast<const uint16_t*>(mask_bias);
@@ -820,7 +836,7 @@ int launch_bwd(int dev, bool tensor_core, const void* Q, const void* K, const vo
 #undef EVO_BWD_TRI
     }
 #define EVO_BWD_SIMT(T)                                                                                         \
-    return launch_bwd_simt<T>(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair, workspace, B, \
+    return launch_bwd_simt<T>(dev, Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair, workspace, B, \
                               N, S, H, D, st)
     if (dtype == EVO_DTYPE_FP32) EVO_BWD_SIMT(float);
     if (dtype == EVO_DTYPE_FP16) EVO_BWD_SIMT(__half);
