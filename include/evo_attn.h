@@ -70,8 +70,10 @@ typedef enum {
     EVO_ERR_MISALIGNED        = -4,  /* a pointer breaks the alignment rule    */
     EVO_ERR_CUDA              = -5,  /* a CUDA runtime/driver call failed      */
     EVO_ERR_TIMEOUT           = -6,  /* a device-side wait gave up (see above) */
-    EVO_ERR_RANGE             = -7   /* an input value is outside the range the
+    EVO_ERR_RANGE             = -7,  /* an input value is outside the range the
                                         kernel's arithmetic supports (see below) */
+    EVO_ERR_SCRATCH           = -8   /* evo_attn_bwd_noalloc: the problem needs more
+                                        scratch than the library's static array holds */
 } evo_status_t;
 
 /*
@@ -245,6 +247,43 @@ EVO_API int evo_attn_bwd(const void* Q, const void* K, const void* V,
                  const void* O, const float* LSE, const void* dO,
                  void* dQ, void* dK, void* dV, void* dmask, void* dpair,
                  void* workspace, int64_t workspace_bytes,
+                 int64_t B, int64_t N, int64_t S, int64_t H, int64_t D,
+                 int dtype, evo_stream_t stream);
+
+/*
+ * evo_attn_bwd_noalloc — evo_attn_bwd without a caller workspace: the
+ * scratch is a static array of EVO_ATTN_NOALLOC_SCRATCH_BYTES (64 MiB) per
+ * device inside this library, so the call allocates no memory of any kind.
+ * The guide has no counterpart; this is an interface of this library.
+ *
+ * For callers that cannot allocate device memory at the point of the call:
+ * a process that has handed all of the device's memory to a pool of its own
+ * (so that a new allocation would fail or fragment it), or code that must
+ * not bring in the device-wide synchronisation that releasing device memory
+ * (cudaFree) implies.  Everything else is as for evo_attn_bwd (arguments
+ * without workspace / workspace_bytes, envelope, status codes, gradients).
+ *
+ *  - Size limit: evo_attn_bwd_workspace_size(B, N, S, H, D) must not exceed
+ *    EVO_ATTN_NOALLOC_SCRATCH_BYTES, else EVO_ERR_SCRATCH is returned and
+ *    nothing is launched (e.g. B=1, N=64, S=256, H=4, D=32 needs 10.0 MB;
+ *    N=S=384, H=4, D=32 needs 83 MB and is refused).
+ *  - Setup: the first call on a device looks up the array's device address
+ *    (once per device, with that device current) and keeps it; make that
+ *    first call before any stream capture on the device.
+ *  - Zeroing: the call itself clears, on `stream`, the parts of the scratch
+ *    that must start at zero (the fp32 sums of dQ, dmask and dpair and a
+ *    work-list counter); no other part needs to start at zero, and nothing
+ *    of one call is read by the next.
+ *  - Concurrency: every call on a device uses the same array.  Calls whose
+ *    work overlaps on the device (on different streams without ordering
+ *    between them, or from several host threads) race on it and give wrong
+ *    gradients; order them (one stream, or events).
+ */
+#define EVO_ATTN_NOALLOC_SCRATCH_BYTES (64ll << 20)
+EVO_API int evo_attn_bwd_noalloc(const void* Q, const void* K, const void* V,
+                 const void* mask_bias, const void* pair_bias,
+                 const void* O, const float* LSE, const void* dO,
+                 void* dQ, void* dK, void* dV, void* dmask, void* dpair,
                  int64_t B, int64_t N, int64_t S, int64_t H, int64_t D,
                  int dtype, evo_stream_t stream);
 

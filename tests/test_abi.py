@@ -40,7 +40,7 @@ def test_exports_match_header(lib):
 
 
 def test_strerror_and_version(lib):
-    for code in range(-7, 1):
+    for code in range(-8, 1):
         s = evo.evo_attn_strerror(code)
         assert s and s != "unknown status"
     assert evo.evo_attn_strerror(-99) == "unknown status"

@@ -28,7 +28,8 @@ __all__ = [
     "EvoAttnError", "library_path", "load_library",
     "EVO_DTYPE_BF16", "EVO_DTYPE_FP32", "EVO_DTYPE_FP16",
     "EVO_OK", "EVO_ERR_INVALID_ARG", "EVO_ERR_UNSUPPORTED_DTYPE", "EVO_ERR_UNSUPPORTED_SHAPE",
-    "EVO_ERR_MISALIGNED", "EVO_ERR_CUDA", "EVO_ERR_TIMEOUT", "EVO_ERR_RANGE",
+    "EVO_ERR_MISALIGNED", "EVO_ERR_CUDA", "EVO_ERR_TIMEOUT", "EVO_ERR_RANGE", "EVO_ERR_SCRATCH",
+    "evo_attn_bwd_noalloc", "NOALLOC_SCRATCH_BYTES",
 ]
 
 EVO_DTYPE_BF16 = 0
@@ -43,6 +44,10 @@ EVO_ERR_MISALIGNED = -4
 EVO_ERR_CUDA = -5
 EVO_ERR_TIMEOUT = -6
 EVO_ERR_RANGE = -7
+EVO_ERR_SCRATCH = -8
+
+# size of the static scratch behind evo_attn_bwd_noalloc (EVO_ATTN_NOALLOC_SCRATCH_BYTES)
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libevoattn.so")
@@ -88,6 +93,8 @@ def load_library():
     lib.evo_attn_bwd_workspace_size.restype = i64
     lib.evo_attn_bwd.argtypes = [vp] * 14 + [i64, i64, i64, i64, i64, i64, i32, vp]
     lib.evo_attn_bwd.restype = i32
+    lib.evo_attn_bwd_noalloc.argtypes = [vp] * 13 + [i64, i64, i64, i64, i64, i32, vp]
+    lib.evo_attn_bwd_noalloc.restype = i32
     _lib = lib
     return lib
 
@@ -134,6 +141,14 @@ def evo_attn_bwd(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, d
     """The C backward entry point with raw addresses (ints); returns the status code."""
     return int(load_library().evo_attn_bwd(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair,
                                            workspace, workspace_bytes, B, N, S, H, D, dtype, stream))
+
+
+def evo_attn_bwd_noalloc(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair,
+                         B: int, N: int, S: int, H: int, D: int, dtype: int, stream: Optional[int]) -> int:
+    """The C backward entry point that uses the library's static scratch (no
+    workspace argument, no allocation); raw addresses; returns the status code."""
+    return int(load_library().evo_attn_bwd_noalloc(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask,
+                                                   dpair, B, N, S, H, D, dtype, stream))
 
 
 def _ptr(t: Optional[torch.Tensor]):

@@ -453,6 +453,7 @@ extern "C" EVO_API const char* evo_attn_strerror(int status) {
         case EVO_ERR_CUDA: return "a CUDA call failed";
         case EVO_ERR_TIMEOUT: return "a device-side wait timed out";
         case EVO_ERR_RANGE: return "an input value is outside the supported range (|V| > 65504 with bf16, or a non-finite output)";
+        case EVO_ERR_SCRATCH: return "the problem needs more scratch than the static backward scratch holds (64 MiB)";
         default: return "unknown status";
     }
 }
@@ -872,4 +873,67 @@ extern "C" EVO_API int evo_attn_bwd(const void* Q, const void* K, const void* V,
         if (ptr != nullptr && device_of(ptr) != dev) return EVO_ERR_INVALID_ARG;
     return launch_bwd(dev, tensor_core, Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair,
                       workspace, B, N, S, H, D, dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------- backward without allocation
+
+// Scratch of evo_attn_bwd_noalloc: one static array per device, created when
+// the library is loaded, so the entry point never allocates.
+static __device__ __align__(256) unsigned char g_bwd_scratch[EVO_ATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+// The array's device address on `dev` (the current device), looked up on the
+// first call for that device and kept.
+int noalloc_scratch(int dev, void** out) {
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return EVO_ERR_CUDA;
+        }
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return EVO_OK;
+}
+
+}  // namespace
+
+extern "C" EVO_API int evo_attn_bwd_noalloc(const void* Q, const void* K, const void* V, const void* mask_bias,
+                                            const void* pair_bias, const void* O, const float* LSE, const void* dO,
+                                            void* dQ, void* dK, void* dV, void* dmask, void* dpair, int64_t B,
+                                            int64_t N, int64_t S, int64_t H, int64_t D, int dtype,
+                                            evo_stream_t stream) {
+    if (B < 0 || N < 0 || S < 0 || H < 0 || D < 0) return EVO_ERR_INVALID_ARG;
+    if (B == 0 || N == 0 || S == 0 || H == 0) {
+        bool unused = false;  // the checks of an empty call, without a workspace to name
+        return check_bwd(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair, nullptr, 0, B, N, S,
+                         H, D, dtype, &unused);
+    }
+    BwdLayout L;
+    if (!bwd_layout(B, N, S, H, D, &L)) return EVO_ERR_UNSUPPORTED_SHAPE;
+    if (L.total > EVO_ATTN_NOALLOC_SCRATCH_BYTES) return EVO_ERR_SCRATCH;
+    if (!Q) return EVO_ERR_INVALID_ARG;
+    RelaxedCapture relaxed;
+    DeviceScope scope;
+    const int dev = select_device_of(Q, scope);
+    if (dev < 0) return dev;
+    if (dev >= kMaxDevices) return EVO_ERR_UNSUPPORTED_SHAPE;
+    void* scratch = nullptr;
+    const int sst = noalloc_scratch(dev, &scratch);
+    if (sst != EVO_OK) return sst;
+    bool tensor_core = false;
+    const int st = check_bwd(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair, scratch,
+                             EVO_ATTN_NOALLOC_SCRATCH_BYTES, B, N, S, H, D, dtype, &tensor_core);
+    if (st != EVO_OK) return st;
+    for (const void* ptr : {K, V, O, static_cast<const void*>(LSE), mask_bias, pair_bias, dO,
+                            static_cast<const void*>(dQ), static_cast<const void*>(dK), static_cast<const void*>(dV),
+                            static_cast<const void*>(dmask), static_cast<const void*>(dpair)})
+        if (ptr != nullptr && device_of(ptr) != dev) return EVO_ERR_INVALID_ARG;
+    return launch_bwd(dev, tensor_core, Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair, scratch,
+                      B, N, S, H, D, dtype, reinterpret_cast<cudaStream_t>(stream));
 }
