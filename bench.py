@@ -274,7 +274,7 @@ def workload_config(wl, flush=False):
 def pair_bias_stream(wl) -> int:
     """Bytes of pair-bias tiles loaded per launch (0 without a pair bias, or
     when S % 8 != 0 and the softmax reads the bias from global memory)."""
-    if wl.name == "msa_col_2048" or wl.dtype == torch.float32 or wl.S % 8:
+    if wl.name.startswith("msa_col") or wl.dtype == torch.float32 or wl.S % 8:
         return 0
     ns = 3 if wl.D <= 32 else (2 if wl.D == 64 else 1)
     qb = (wl.S + 127) // 128
@@ -285,7 +285,7 @@ def pair_bias_stream(wl) -> int:
 def alg_bytes(wl) -> int:
     es = 2 if wl.dtype == torch.bfloat16 else 4
     qkvo = 4 * wl.B * wl.N * wl.S * wl.H * wl.D * es
-    pair = wl.B * wl.H * wl.S * wl.S * es if wl.name != "msa_col_2048" else 0
+    pair = wl.B * wl.H * wl.S * wl.S * es if not wl.name.startswith("msa_col") else 0
     mask = wl.B * wl.N * wl.S * es
     lse = wl.B * wl.N * wl.H * wl.S * 4
     return qkvo + pair + mask + lse

@@ -20,8 +20,13 @@
 //     dQ      = dT K        (MMA, M = 128 queries, N = D), added to an fp32
 //                            accumulator in global memory (every key block of
 //                            the slice contributes)
-//     dpair  += dT          (fp32 vector reductions into global memory: the
-//                            pair bias is shared by every n)
+//     dpair  += dT          (fp32, into global memory: the pair bias is shared
+//                            by every n)
+//
+// Both global sums are TMA tile reductions (cp.reduce.async.bulk.tensor
+// .add): a warp stages its 32 rows in shared memory and one lane issues the
+// reduction, so L2 adds whole 128 B (dpair) or 64 B (dQ) rows instead of the
+// 16 B pieces of per-thread vector atomics.
 //
 // dK and dV stay in tensor memory for the whole unit and are written once; the
 // fp32 dQ, dmask and dpair sums are rounded to the output type by a final
@@ -89,7 +94,15 @@ struct BwdCfg {
     static constexpr int OFF_P = OFF_PAIR + PAIR_STAGES * PAIR_BYTES;
     static constexpr int OFF_DT = OFF_P + PT_BYTES;
     static constexpr int OFF_MASK = OFF_DT + PT_BYTES;  // [2][128] f32: (mask - c) log2(e) per key
-    static constexpr int OFF_BAR = OFF_MASK + 2 * kBN * 4;
+    // per softmax warp: 32 rows x 32 fp32 of dT (128 B rows, 128 B swizzle),
+    // added to dpair by one TMA tile reduction
+    static constexpr int STG_WARP = 32 * 128;
+    static constexpr int OFF_STG = OFF_MASK + 2 * kBN * 4;
+    // per dQ warp: 32 rows x 16 fp32 of dQ (64 B rows, 64 B swizzle), added to
+    // the fp32 dQ sums by TMA tile reductions, 16 columns at a time
+    static constexpr int QSTG_WARP = 32 * 64;
+    static constexpr int OFF_QSTG = OFF_STG + (HAS_PAIR ? 4 * STG_WARP : 0);
+    static constexpr int OFF_BAR = OFF_QSTG + 4 * QSTG_WARP;
     static constexpr int BAR_KVF = 0;                            // [KV_STAGES] K, V landed
     static constexpr int BAR_KVE = BAR_KVF + KV_STAGES;          // [KV_STAGES] last MMA of the unit done
     static constexpr int BAR_QF = BAR_KVE + KV_STAGES;           // [2] Q, dO landed
@@ -170,7 +183,8 @@ template <int D, bool HAS_PAIR, bool F16>
 __global__ void __launch_bounds__(BwdCfg<D, HAS_PAIR, F16>::THREADS, 1)
 evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                   const __grid_constant__ CUtensorMap tm_pair, const BwdTriParams p) {
+                   const __grid_constant__ CUtensorMap tm_pair, const __grid_constant__ CUtensorMap tm_dpair,
+                   const __grid_constant__ CUtensorMap tm_dq, const BwdTriParams p) {
     using C = BwdCfg<D, HAS_PAIR, F16>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -414,17 +428,49 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         float* mask_w = reinterpret_cast<float*>(smem + C::OFF_MASK);
         bool ok = true;
         int uc = 0, g = 0;
+        // Global loads are issued one step (rows) or one unit (mask) ahead of
+        // their use, so that their latency hides behind a step's work.
+        auto row_loads = [&](const BwdUnit& t, int qb, float& lr, float& dl) {
+            const int i = qb * kBM + r;
+            lr = INFINITY;
+            dl = 0.f;
+            if (i < p.S) {
+                const size_t ri = (size_t(t.bn) * p.H + t.h) * p.S + i;
+                lr = __ldg(p.lse_r + ri);
+                dl = __ldg(p.delta + ri);
+            }
+        };
+        auto mask_loads = [&](const BwdUnit& t, uint32_t& mbits, float& c) {
+            const int j = t.kb * kBN + r;
+            mbits = 0u;
+            c = 0.f;
+            if (p.mask != nullptr && j < p.S) {
+                mbits = p.mask[size_t(t.bn) * p.S + j];
+                c = __ldg(p.cmask + t.bn);
+            }
+        };
+        float lr_n = INFINITY, dl_n = 0.f, c_n = 0.f;
+        uint32_t mbits_n = 0u;
+        if (int(blockIdx.x) < p.num_units) {
+            const BwdUnit t0 = bwd_unit(p, blockIdx.x);
+            row_loads(t0, 0, lr_n, dl_n);
+            mask_loads(t0, mbits_n, c_n);
+        }
         for (int u = blockIdx.x; u < p.num_units && ok; u += G, ++uc) {
             const BwdUnit t = bwd_unit(p, u);
+            const bool has_next_unit = u + G < p.num_units;
+            const BwdUnit tn = bwd_unit(p, has_next_unit ? u + G : u);
             const int mb = uc & 1;
             {
                 // this unit's key block of the mask row: (mask - c) log2(e), -inf past S
                 // or more than kMaskFloor below c (such a weight is exactly zero)
                 const int j = t.kb * kBN + r;
+                const uint32_t mbits = mbits_n;
+                const float cm = c_n;
+                if (has_next_unit) mask_loads(tn, mbits_n, c_n);
                 float ml = -INFINITY;
                 if (j < p.S) {
-                    float x = 0.f;
-                    if (p.mask != nullptr) x = bits_to_f32<F16>(p.mask[size_t(t.bn) * p.S + j]) - p.cmask[t.bn];
+                    const float x = (p.mask != nullptr) ? bits_to_f32<F16>(mbits) - cm : 0.f;
                     ml = (x < -kMaskFloor) ? -INFINITY : x * kLog2e;
                 }
                 mask_w[mb * kBN + r] = ml;
@@ -435,26 +481,19 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             }
             const float* ml2 = mask_s + mb * kBN;
             for (int qb = 0; qb < nqb; ++qb, ++g) {
-                const int i = qb * kBM + r;
-                float lse2 = INFINITY, dl = 0.f;
-                if (i < p.S) {
-                    const size_t ri = (size_t(t.bn) * p.H + t.h) * p.S + i;
-                    const float lr = __ldg(p.lse_r + ri);
-                    lse2 = (lr == INFINITY) ? INFINITY : lr * kLog2e;
-                    dl = __ldg(p.delta + ri);
-                }
+                const float lr = lr_n, dl = dl_n;
+                if (qb + 1 < nqb) row_loads(t, qb + 1, lr_n, dl_n);
+                else if (has_next_unit) row_loads(tn, 0, lr_n, dl_n);
                 ok = wait_warp(bar(C::BAR_SF), uint32_t(g) & 1u, abort_flag);
                 if (!ok) break;
                 ptx::tc_fence_after();
+                const float lse2 = (lr == INFINITY) ? INFINITY : lr * kLog2e;
                 const int ps = HAS_PAIR ? g % C::PAIR_RING : 0;
                 if constexpr (HAS_PAIR) {
                     ok = wait_warp(bar(C::BAR_BF + ps), uint32_t(g / C::PAIR_RING) & 1u, abort_flag);
                     if (!ok) break;
                 }
                 const uint32_t ptile = sb + C::OFF_PAIR + uint32_t(ps * C::PAIR_BYTES);
-                float* dpair_row = (p.dpair_acc != nullptr && i < p.S)
-                                       ? p.dpair_acc + ((size_t(t.b) * p.H + t.h) * p.S + i) * size_t(p.S)
-                                       : nullptr;
 #pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     float s[32], dp[32];
@@ -513,13 +552,29 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         ptx::st_shared_v4(sb + C::OFF_DT + off,
                                           make_uint4(dw[4 * u4], dw[4 * u4 + 1], dw[4 * u4 + 2], dw[4 * u4 + 3]));
                     }
-                    if (dpair_row != nullptr) {
-                        const int j0 = t.kb * kBN + 32 * c;
+                    if (HAS_PAIR && p.dpair_acc != nullptr) {
+                        // this warp's 32 rows x 32 keys of dT, staged in shared memory and
+                        // added to dpair by one TMA tile reduction (whole 128 B rows in L2);
+                        // lane 0 issues it and first waits until the previous one has
+                        // read the stage
+                        const uint32_t stg = sb + C::OFF_STG + uint32_t(wq * C::STG_WARP);
+                        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                        __syncwarp();
 #pragma unroll
                         for (int q4 = 0; q4 < 8; ++q4)
-                            if (j0 + 4 * q4 < p.S)
-                                red_add_v4(dpair_row + j0 + 4 * q4, dp[4 * q4], dp[4 * q4 + 1], dp[4 * q4 + 2],
-                                           dp[4 * q4 + 3]);
+                            ptx::st_shared_v4(stg + swz_chunk<128>(lane, q4),
+                                              make_uint4(__float_as_uint(dp[4 * q4]), __float_as_uint(dp[4 * q4 + 1]),
+                                                         __float_as_uint(dp[4 * q4 + 2]), __float_as_uint(dp[4 * q4 + 3])));
+                        ptx::fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            asm volatile(
+                                "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+                                " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(&tm_dpair)),
+                                "r"(stg), "r"(t.kb * kBN + 32 * c), "r"(qb * kBM + 32 * wq), "r"(t.b * p.H + t.h)
+                                : "memory");
+                            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                        }
                     }
                 }
                 if (!ok) break;
@@ -532,6 +587,9 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ptx::mbar_arrive_elect(bar(C::BAR_PF));
             }
         }
+        // every dpair reduction of this warp has been carried out
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        __syncwarp();
         if (!ok) aborted = true;
     } else if (warp >= 8) {
         // ------------------------------------------- dQ, dK, dV, dmask out
@@ -559,11 +617,30 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 for (int d0 = LDW; d0 < D; d0 += 32) ptx::reg_fence_x32(reinterpret_cast<uint32_t*>(dq + d0));
                 ptx::tc_fence_before();
                 ptx::mbar_arrive_elect(bar(C::BAR_DQE));
-                const int i = qb * kBM + r;
-                if (i < p.S) {
-                    float* dst = p.dq_acc + ((size_t(t.bn) * p.S + i) * p.H + t.h) * D;
+                // this warp's 32 rows of dQ into the fp32 sums, 16 columns per TMA
+                // tile reduction (rows past S are clipped by the tensor map)
+                const uint32_t stg = sb + C::OFF_QSTG + uint32_t(we * C::QSTG_WARP);
 #pragma unroll
-                    for (int d = 0; d < D; d += 4) red_add_v4(dst + d, dq[d], dq[d + 1], dq[d + 2], dq[d + 3]);
+                for (int x = 0; x < D / 16; ++x) {
+                    if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                    __syncwarp();
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        ptx::st_shared_v4(stg + swz_chunk<64>(lane, q4),
+                                          make_uint4(__float_as_uint(dq[16 * x + 4 * q4]),
+                                                     __float_as_uint(dq[16 * x + 4 * q4 + 1]),
+                                                     __float_as_uint(dq[16 * x + 4 * q4 + 2]),
+                                                     __float_as_uint(dq[16 * x + 4 * q4 + 3])));
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        asm volatile(
+                            "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group"
+                            " [%0, {%2, %3, %4, %5}], [%1];" ::"l"(reinterpret_cast<uint64_t>(&tm_dq)),
+                            "r"(stg), "r"(16 * x), "r"(t.h), "r"(qb * kBM + 32 * we), "r"(int(t.bn))
+                            : "memory");
+                        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                    }
                 }
             }
             if (!ok) break;
@@ -613,6 +690,9 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (p.dmask_acc != nullptr) atomicAdd(p.dmask_acc + size_t(t.bn) * p.S + j, dka[D]);
             }
         }
+        // every dQ reduction of this warp has been carried out
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        __syncwarp();
         if (!ok) aborted = true;
     }
     (void)aborted;

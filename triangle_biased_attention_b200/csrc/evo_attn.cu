@@ -755,8 +755,9 @@ int launch_bwd_tri(int dev, const void* Q, const void* K, const void* V, const v
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
         return EVO_ERR_CUDA;
     const CUtensorMapDataType dt = F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    CUtensorMap tq, tk, tv, tdo, tp;
+    CUtensorMap tq, tk, tv, tdo, tp, tdp, tdq;
     std::memset(&tp, 0, sizeof(tp));
+    std::memset(&tdp, 0, sizeof(tdp));
     if (!encode_qkv(&tq, Q, B * N, S, H, D, 16, dt) || !encode_qkv(&tk, K, B * N, S, H, D, 16, dt) ||
         !encode_qkv(&tv, V, B * N, S, H, D, 16, dt) || !encode_qkv(&tdo, dO, B * N, S, H, D, 16, dt))
         return EVO_ERR_CUDA;
@@ -774,6 +775,31 @@ int launch_bwd_tri(int dev, const void* Q, const void* K, const void* V, const v
                                                     dpair, workspace, B, N, S, H, D);
     if (launch_rowstats<T>(dev, bp, B, N, S, H, st) != EVO_OK) return EVO_ERR_CUDA;
 
+    if (HAS_PAIR && dpair) {
+        // the fp32 dpair sums as a 3-D tensor {S (key), S (query), B*H}; a box
+        // is 32 keys x 32 queries (128 B rows, 128 B swizzle), the tile one
+        // softmax warp reduces into it per 32-key chunk
+        const cuuint64_t dims[3] = {cuuint64_t(S), cuuint64_t(S), cuuint64_t(B * H)};
+        const cuuint64_t strides[2] = {cuuint64_t(S * 4), cuuint64_t(S * S * 4)};
+        const cuuint32_t box[3] = {32, 32, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (encode_fn()(&tdp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ws + L.dpair_acc, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return EVO_ERR_CUDA;
+    }
+    {
+        // the fp32 dQ sums as a 4-D tensor {D, H, S, B*N} like Q; a box is 16
+        // columns of 32 rows (64 B rows, 64 B swizzle)
+        const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(S), cuuint64_t(B * N)};
+        const cuuint64_t strides[3] = {cuuint64_t(D * 4), cuuint64_t(H * D * 4), cuuint64_t(S * H * D * 4)};
+        const cuuint32_t box[4] = {16, 1, 32, 1};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        if (encode_fn()(&tdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ws + L.dq_acc, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return EVO_ERR_CUDA;
+    }
     evo::BwdTriParams p;
     p.mask = static_cast<const uint16_t*>(mask_bias);
     p.cmask = bp.cmask;
@@ -797,7 +823,7 @@ int launch_bwd_tri(int dev, const void* Q, const void* K, const void* V, const v
     cfg.blockDim = dim3(C::THREADS, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = st;
-    if (cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, tdo, tp, p) != cudaSuccess) return EVO_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kernel, tq, tk, tv, tdo, tp, tdp, tdq, p) != cudaSuccess) return EVO_ERR_CUDA;
 
     cudaLaunchConfig_t pc = {};
     const long long work = std::max(n_q / 4, std::max(dmask ? n_m : 0ll, dpair ? n_p : 0ll));

@@ -24,6 +24,11 @@ residue counts the other pages discuss):
                 masked, plus 2 fully masked n
   tri_1024      B=1 N=1024 S=1024 H=4 D=32 bf16 (D=64 variant: tri_1024_d64),
                 pair N(0,1) with 1% of entries set to +8, tail of 0..64 masked
+Smaller cases of the same kernels, for single-launch profiler captures
+(inputs still larger than the 126 MB L2):
+  msa_col_512   B=1 N=256 S=512 H=8 D=32 bf16, no pair, per-n tail of 0..128
+                masked, plus 1 fully masked n
+  tri_512_d64   B=1 N=512 S=512 H=4 D=64 bf16, generated like tri_1024
 """
 from __future__ import annotations
 
@@ -90,6 +95,10 @@ WORKLOADS = {
                              "large triangle attention, N_res=1024, D=64"),
     "tri_512_d128": Workload("tri_512_d128", 1, 512, 512, 4, 128, torch.bfloat16,
                              "triangle attention, N_res=512, D=128 (head-dim envelope)"),
+    "msa_col_512": Workload("msa_col_512", 1, 256, 512, 8, 32, torch.bfloat16,
+                            "MSA column-wise attention, mask only, 512 sequences (profiling size)"),
+    "tri_512_d64": Workload("tri_512_d64", 1, 512, 512, 4, 64, torch.bfloat16,
+                            "triangle attention, N_res=512, D=64 (profiling size)"),
 }
 
 
@@ -139,17 +148,17 @@ def make_case(name: str, seed: int = 0) -> Case:
     elif name == "msa_row_512":
         pair = _normal(rng, (B, 1, H, S, S), std=float(np.sqrt(2.0)))
         keep = rng.random((B, N, S)) >= 0.05
-    elif name == "msa_col_2048":
-        tails = rng.integers(0, 513, size=(B, N))
+    elif name in ("msa_col_2048", "msa_col_512"):
+        tails = rng.integers(0, S // 4 + 1, size=(B, N))
         for b in range(B):
             for n in range(N):
                 t = int(tails[b, n])
                 if t:
                     keep[b, n, S - t:] = False
-        full = rng.choice(N, size=2, replace=False)
+        full = rng.choice(N, size=2 if name == "msa_col_2048" else 1, replace=False)
         keep[:, full, :] = False
         meta["fully_masked_n"] = sorted(int(x) for x in full)
-    elif name in ("tri_1024", "tri_1024_d64", "tri_512_d128"):
+    elif name in ("tri_1024", "tri_1024_d64", "tri_512_d128", "tri_512_d64"):
         pair = _normal(rng, (B, 1, H, S, S))
         spikes = rng.random((B, 1, H, S, S)) < 0.01
         pair[spikes] = np.float32(8.0)
