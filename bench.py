@@ -40,6 +40,8 @@ from triangle_biased_attention_b200 import workloads as W  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 KERNEL_SOURCES = ["common.cuh", "ptx_sm100.cuh", "tile_sm100.cuh", "fwd_tri_sm100.cuh", "evo_attn.cu"]
+KERNEL_SOURCES_BWD = ["common.cuh", "ptx_sm100.cuh", "tile_sm100.cuh", "bwd_simt.cuh", "bwd_tri_sm100.cuh",
+                      "evo_attn.cu"]
 KERNEL_NAME = "evo_fwd_tri_kernel"
 
 
@@ -100,23 +102,24 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in (KERNEL_SOURCES if sources is None else sources):
         with open(os.path.join(ROOT, "triangle_biased_attention_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source (else None)."""
+def recorded_traffic(workload: str, sources=None):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary (key: the workload, "bwd:<workload>" for the backward), if it was
+    taken on the current kernel sources (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
         e = d[workload]
-        if e.get("kernel_source_hash") == kernel_source_hash():
+        if e.get("kernel_source_hash") == kernel_source_hash(sources):
             return float(e["dram_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
         pass
@@ -515,7 +518,8 @@ def run_ours_bwd(args, rank, world, local):
     peaks, peak_src = load_peaks()
     achieved = flops / (ms / args.steps * 1e-3) / 1e12
     roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+            "frac": achieved / peaks["bf16_tflops"],
+            "traffic": recorded_traffic("bwd:" + args.workload, KERNEL_SOURCES_BWD),
             "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst figure)" if peak_src == "measured"
             else "fallback (6.65 TB/s, 1.59 PFLOP/s)",
             "alg_flops_per_launch": flops,
