@@ -98,6 +98,11 @@ def test_bwd_fp16_tensor_cores():
     compare(case, 10, "fp16 D=32 tensor cores, no biases")
 
 
+def test_bwd_fp16_d16_tensor_cores():
+    case = W.random_case(2, 3, 200, 2, 16, torch.float16, seed=14, mask="head", pair=True)
+    compare(case, 14, "fp16 D=16 tensor cores")
+
+
 def test_bwd_fp16_fully_masked_rows_are_empty():
     # in fp16 the guide's -1e9 mask is -inf: a fully masked n has no softmax
     # and gets zero gradients
@@ -157,3 +162,25 @@ def test_bwd_tri_1024_sampled():
     ref_p = orc.pair_grad_rows(case.q, case.k, case.v, case.mask, case.pair, do, rows, chunk=128)
     got_p = np.stack([got["dpair"][b, 0, h, i].double().numpy() for (b, h, i) in rows])
     check_grads({"dpair": got_p}, {"dpair": ref_p}, case.dtype, "tri_1024 dpair rows")
+
+
+def test_bwd_msa_col_2048_sampled():
+    """The backward at the full column-attention size (no pair bias; two n
+    whose every key is masked, whose rows take the recomputed LSE): dQ, dK,
+    dV of sampled slices including both fully masked n, and dmask of them."""
+    case = W.make_case("msa_col_2048", 0)
+    do = _upstream(case, 0)
+    got = run_bwd(case, do)
+    orc = oracle.default()
+    B, N, S, H, D = case.shape
+    full = case.meta["fully_masked_n"]
+    slices = [(0, full[0], 0), (0, full[1], 5), (0, 17, 3), (0, 200, 7)]
+    dq, dk, dv, _ = orc.attention_bwd_slices(case.q, case.k, case.v, case.mask, case.pair, do, slices)
+    pick = lambda g: np.stack([g[b, n, :, h, :].double().numpy() for (b, n, h) in slices])
+    check_grads({"dq": pick(got["dq"]), "dk": pick(got["dk"]), "dv": pick(got["dv"])},
+                {"dq": dq, "dk": dk, "dv": dv}, case.dtype, "msa_col_2048 sampled slices")
+    for n in (full[0], 17):
+        hs = [(0, n, h) for h in range(H)]
+        _, _, _, cs = orc.attention_bwd_slices(case.q, case.k, case.v, case.mask, case.pair, do, hs)
+        check_grads({"dmask": got["dmask"][0, n, 0, 0].double().numpy()}, {"dmask": cs.sum(axis=0)},
+                    case.dtype, f"msa_col_2048 dmask n={n}")
