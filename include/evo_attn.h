@@ -1,6 +1,7 @@
 /*
  * evo_attn.h — C ABI of the B200 (sm_100a) biased-attention library,
- * libevoattn.so: the forward pass and its backward pass.
+ * libevoattn.so: the forward pass, its backward pass, and the
+ * triangle-multiplication contraction.
  *
  * The operation is the forward pass that the DeepSpeed DS4Sci_EvoformerAttention
  * guide (hmyw.cn) describes for the four Evoformer attention variants (its
@@ -286,6 +287,47 @@ EVO_API int evo_attn_bwd_noalloc(const void* Q, const void* K, const void* V,
                  void* dQ, void* dK, void* dV, void* dmask, void* dpair,
                  int64_t B, int64_t N, int64_t S, int64_t H, int64_t D,
                  int dtype, evo_stream_t stream);
+
+/*
+ * evo_trimul_workspace_size — bytes of device workspace evo_trimul needs
+ * (three [Bt*C, N, Np] copies, Np = N rounded up to a multiple of 8), or a
+ * negative evo_status_t for negative sizes or byte counts past int64.
+ */
+EVO_API int64_t evo_trimul_workspace_size(int64_t Bt, int64_t N, int64_t C);
+
+/*
+ * evo_trimul — triangle multiplication: the contraction over the third node
+ * of two edge representations, channel by channel.
+ *
+ * The NVIDIA cuEquivariance blog (open-lab.net, "Accelerated molecular
+ * modeling with NVIDIA cuEquivariance and NVIDIA NIM microservices", the
+ * triangle-operations sections) names triangle multiplication beside
+ * triangle attention as the two O(N^3) operations of these models, from
+ * "triangular relationships" (i close to k and k close to j relate i and j),
+ * without a formula.  This library's reading, for every b and channel c:
+ *     outgoing (outgoing = 1):  Z[b,i,j,c] = sum_k A[b,i,k,c] * B[b,j,k,c]
+ *     incoming (outgoing = 0):  Z[b,i,j,c] = sum_k A[b,k,i,c] * B[b,k,j,c]
+ * (the projections, gates and norms around it in a model are per-edge and
+ * not part of this call).
+ *
+ *   A, B       [Bt, N, N, C] of `dtype`, contiguous, 2-byte aligned.
+ *   Z          [Bt, N, N, C] of `dtype`, written (fp32 accumulation, rounded
+ *              to nearest even); must not overlap A, B or the workspace.
+ *   workspace  device scratch of at least evo_trimul_workspace_size(Bt, N, C)
+ *              bytes, 256-byte aligned, owned by the caller, overwritten.
+ *   Bt, N, C   >= 0 (a zero size is a no-op that returns EVO_OK).
+ *   dtype      EVO_DTYPE_BF16 or EVO_DTYPE_FP16 (else EVO_ERR_UNSUPPORTED_DTYPE).
+ *   stream     CUDA stream of the call.
+ *
+ * Three kernels on `stream`: A and B transposed to channel-first copies in
+ * the workspace, a tcgen05 batched GEMM over the Bt*C channel matrices, and
+ * the result transposed back.  Returns EVO_OK once enqueued, or a negative
+ * evo_status_t (EVO_ERR_INVALID_ARG also for a workspace that is too small).
+ * The pages have no interface for this operation; the call follows the shape
+ * conventions of evo_attn_fwd.
+ */
+EVO_API int evo_trimul(const void* A, const void* B, void* Z, void* workspace, int64_t workspace_bytes,
+               int64_t Bt, int64_t N, int64_t C, int outgoing, int dtype, evo_stream_t stream);
 
 /*
  * evo_attn_sync_status — synchronise `stream`, then return and clear the

@@ -239,3 +239,21 @@ def test_backward_wrapper_validates_before_calling():
         evo.evo_attn_backward(q, q, q, None, None, q, lse, q, need_dmask=True)
     with pytest.raises(TypeError):
         evo.evo_attn_backward(q, q, q, None, None, q, lse.double(), q)
+
+
+def test_trimul_checks_arguments(lib):
+    size = evo.evo_trimul_workspace_size(1, 37, 3)
+    assert size == 3 * ((2 * 1 * 3 * 37 * 40 + 255) // 256 * 256)      # rows padded to 40
+    assert evo.evo_trimul_workspace_size(-1, 4, 4) == evo.EVO_ERR_INVALID_ARG
+    call = lambda **kw: evo.evo_trimul(kw.get("A", 0x1000000), kw.get("B", 0x2000000), kw.get("Z", 0x3000000),
+                                       kw.get("W", 0x4000000), kw.get("Wb", 1 << 20), kw.get("Bt", 1),
+                                       kw.get("N", 16), kw.get("C", 4), kw.get("out", 1),
+                                       kw.get("dt", evo.EVO_DTYPE_BF16), None)
+    assert call(Bt=0, A=None) == evo.EVO_OK
+    assert call(dt=evo.EVO_DTYPE_FP32) == evo.EVO_ERR_UNSUPPORTED_DTYPE
+    assert call(out=2) == evo.EVO_ERR_INVALID_ARG
+    assert call(A=None) == evo.EVO_ERR_INVALID_ARG
+    assert call(Wb=16) == evo.EVO_ERR_INVALID_ARG                       # workspace too small
+    assert call(W=0x4000010) == evo.EVO_ERR_MISALIGNED
+    assert call(A=0x1000001) == evo.EVO_ERR_MISALIGNED
+    assert call(Z=0x1000000 + 64) == evo.EVO_ERR_INVALID_ARG            # Z over A

@@ -29,7 +29,7 @@ __all__ = [
     "EVO_DTYPE_BF16", "EVO_DTYPE_FP32", "EVO_DTYPE_FP16",
     "EVO_OK", "EVO_ERR_INVALID_ARG", "EVO_ERR_UNSUPPORTED_DTYPE", "EVO_ERR_UNSUPPORTED_SHAPE",
     "EVO_ERR_MISALIGNED", "EVO_ERR_CUDA", "EVO_ERR_TIMEOUT", "EVO_ERR_RANGE", "EVO_ERR_SCRATCH",
-    "evo_attn_bwd_noalloc", "NOALLOC_SCRATCH_BYTES",
+    "evo_attn_bwd_noalloc", "NOALLOC_SCRATCH_BYTES", "evo_trimul", "evo_trimul_workspace_size", "trimul",
 ]
 
 EVO_DTYPE_BF16 = 0
@@ -95,6 +95,10 @@ def load_library():
     lib.evo_attn_bwd.restype = i32
     lib.evo_attn_bwd_noalloc.argtypes = [vp] * 13 + [i64, i64, i64, i64, i64, i32, vp]
     lib.evo_attn_bwd_noalloc.restype = i32
+    lib.evo_trimul_workspace_size.argtypes = [i64, i64, i64]
+    lib.evo_trimul_workspace_size.restype = i64
+    lib.evo_trimul.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i32, i32, vp]
+    lib.evo_trimul.restype = i32
     _lib = lib
     return lib
 
@@ -149,6 +153,17 @@ def evo_attn_bwd_noalloc(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, 
     workspace argument, no allocation); raw addresses; returns the status code."""
     return int(load_library().evo_attn_bwd_noalloc(Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask,
                                                    dpair, B, N, S, H, D, dtype, stream))
+
+
+def evo_trimul_workspace_size(Bt: int, N: int, C: int) -> int:
+    """Workspace bytes of evo_trimul, or a negative status code."""
+    return int(load_library().evo_trimul_workspace_size(Bt, N, C))
+
+
+def evo_trimul(A, B, Z, workspace, workspace_bytes: int, Bt: int, N: int, C: int, outgoing: int, dtype: int,
+               stream: Optional[int]) -> int:
+    """The C triangle-multiplication entry point with raw addresses; returns the status code."""
+    return int(load_library().evo_trimul(A, B, Z, workspace, workspace_bytes, Bt, N, C, outgoing, dtype, stream))
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -326,3 +341,40 @@ def evo_attn_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if status != EVO_OK:
         raise EvoAttnError(status, "evo_attn_bwd")
     return dq, dk, dv, dmask, dpair
+
+
+def trimul(a: torch.Tensor, b: torch.Tensor, outgoing: bool = True, out: Optional[torch.Tensor] = None,
+           workspace: Optional[torch.Tensor] = None,
+           stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Triangle multiplication on CUDA tensors: a, b [Bt, N, N, C] bf16 or fp16,
+    contiguous; returns Z [Bt, N, N, C] with Z[:, i, j] = sum_k a[:, i, k] b[:, j, k]
+    (outgoing) or sum_k a[:, k, i] b[:, k, j] (incoming), channel by channel.
+    ``workspace``: optional uint8 CUDA tensor of ``evo_trimul_workspace_size``
+    bytes (allocated here when not given).  Runs on ``stream`` (default: the
+    current stream) without synchronising."""
+    if a.dim() != 4 or a.shape[1] != a.shape[2]:
+        raise ValueError("a must be [Bt, N, N, C]")
+    if tuple(b.shape) != tuple(a.shape):
+        raise ValueError(f"b has shape {tuple(b.shape)}, expected {tuple(a.shape)}")
+    if a.dtype not in (torch.bfloat16, torch.float16) or b.dtype != a.dtype:
+        raise TypeError("a and b must both be bf16 or both fp16")
+    if a.device.type != "cuda" or b.device != a.device:
+        raise ValueError("a and b must be on one CUDA device")
+    if not (a.is_contiguous() and b.is_contiguous()):
+        raise ValueError("a and b must be contiguous")
+    Bt, N, _, C = a.shape
+    need = evo_trimul_workspace_size(Bt, N, C)
+    if need < 0:
+        raise EvoAttnError(need, "evo_trimul_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=a.device)
+    if out is None:
+        out = torch.empty_like(a)
+    if stream is None:
+        stream = torch.cuda.current_stream(a.device)
+    status = evo_trimul(a.data_ptr(), b.data_ptr(), out.data_ptr(), workspace.data_ptr(),
+                        workspace.numel() * workspace.element_size(), Bt, N, C, 1 if outgoing else 0,
+                        _DTYPES[a.dtype], stream.cuda_stream)
+    if status != EVO_OK:
+        raise EvoAttnError(status, "evo_trimul")
+    return out

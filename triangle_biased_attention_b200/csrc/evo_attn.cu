@@ -25,6 +25,7 @@
 #include "fwd_f32.cuh"
 #include "bwd_simt.cuh"
 #include "bwd_tri_sm100.cuh"
+#include "trimul_sm100.cuh"
 
 namespace {
 
@@ -962,4 +963,134 @@ extern "C" EVO_API int evo_attn_bwd_noalloc(const void* Q, const void* K, const 
         if (ptr != nullptr && device_of(ptr) != dev) return EVO_ERR_INVALID_ARG;
     return launch_bwd(dev, tensor_core, Q, K, V, mask_bias, pair_bias, O, LSE, dO, dQ, dK, dV, dmask, dpair, scratch,
                       B, N, S, H, D, dtype, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------ triangle multiplication
+
+namespace {
+
+// Workspace of evo_trimul: the channel-first copies of A and B and the
+// channel-first result, [Bt*C, N, Np] each (Np = N rounded up to 8), on
+// 256-byte boundaries.
+bool trimul_layout(int64_t Bt, int64_t N, int64_t C, int64_t* section, int64_t* total) {
+    const int64_t np = (N + 7) / 8 * 8;
+    int64_t e, bytes;
+    if (!mul_ok(Bt, C, &e) || !mul_ok(e, N, &e) || !mul_ok(e, np, &e) || !mul_ok(e, 2, &bytes) ||
+        bytes > INT64_MAX / 4)
+        return false;
+    *section = (bytes + 255) / 256 * 256;
+    *total = 3 * *section;
+    return true;
+}
+
+template <bool OUTGOING, bool F16>
+int launch_trimul(int dev, const void* A, const void* Bm, void* Z, void* workspace, int64_t Bt, int64_t N,
+                  int64_t Cc, cudaStream_t st) {
+    using Cfg = evo::TrimulCfg<OUTGOING, F16>;
+    using T = typename std::conditional<F16, __half, uint16_t>::type;
+    auto kernel = evo::evo_trimul_gemm_kernel<OUTGOING, F16>;
+    static AttrOnce attr;
+    if (!attr.ensure(dev, kernel, Cfg::SMEM_BYTES)) return EVO_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return EVO_ERR_CUDA;
+    int64_t section = 0, total = 0;
+    trimul_layout(Bt, N, Cc, &section, &total);  // checked by the caller
+    const int64_t np = (N + 7) / 8 * 8;
+    char* ws = static_cast<char*>(workspace);
+    T* ac = reinterpret_cast<T*>(ws);
+    T* bc = reinterpret_cast<T*>(ws + section);
+    T* zc = reinterpret_cast<T*>(ws + 2 * section);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = st;
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.gridDim = dim3(unsigned(Bt * N), unsigned((N + 31) / 32), unsigned((Cc + 31) / 32));
+    if (cudaLaunchKernelEx(&cfg, evo::evo_trimul_to_cfirst<T>, static_cast<const T*>(A), ac, int(N), int(Cc),
+                           int(np)) != cudaSuccess ||
+        cudaLaunchKernelEx(&cfg, evo::evo_trimul_to_cfirst<T>, static_cast<const T*>(Bm), bc, int(N), int(Cc),
+                           int(np)) != cudaSuccess)
+        return EVO_ERR_CUDA;
+
+    // the channel matrices as a 3-D tensor {N (columns), N (rows), Bt*C}, rows
+    // Np elements apart; a box is 64 x 64 (128 B rows, 128 B swizzle)
+    const CUtensorMapDataType dt = F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint64_t dims[3] = {cuuint64_t(N), cuuint64_t(N), cuuint64_t(Bt * Cc)};
+    const cuuint64_t strides[2] = {cuuint64_t(np * 2), cuuint64_t(N * np * 2)};
+    const cuuint32_t box[3] = {64, 64, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUtensorMap ta, tb;
+    if (encode_fn()(&ta, dt, 3, ac, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        encode_fn()(&tb, dt, 3, bc, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return EVO_ERR_CUDA;
+    evo::TrimulParams p;
+    p.zc = reinterpret_cast<uint16_t*>(zc);
+    p.N = int(N);
+    p.ldz = int(np);
+    p.tiles_mn = int((N + 127) / 128);
+    p.num_tiles = int(Bt * Cc * p.tiles_mn * p.tiles_mn);
+    p.k_steps = int((N + 63) / 64);
+    cudaLaunchConfig_t gc = {};
+    gc.stream = st;
+    gc.blockDim = dim3(Cfg::THREADS, 1, 1);
+    gc.gridDim = dim3(unsigned(p.num_tiles < sms ? p.num_tiles : sms), 1, 1);
+    gc.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    if (cudaLaunchKernelEx(&gc, kernel, ta, tb, p) != cudaSuccess) return EVO_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, evo::evo_trimul_to_clast<T>, static_cast<const T*>(zc), static_cast<T*>(Z),
+                              int(N), int(Cc), int(np)) == cudaSuccess
+               ? EVO_OK
+               : EVO_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" EVO_API int64_t evo_trimul_workspace_size(int64_t Bt, int64_t N, int64_t C) {
+    if (Bt < 0 || N < 0 || C < 0) return EVO_ERR_INVALID_ARG;
+    int64_t section, total;
+    if (!trimul_layout(Bt, N, C, &section, &total)) return EVO_ERR_UNSUPPORTED_SHAPE;
+    return total;
+}
+
+extern "C" EVO_API int evo_trimul(const void* A, const void* Bm, void* Z, void* workspace, int64_t workspace_bytes,
+                                  int64_t Bt, int64_t N, int64_t C, int outgoing, int dtype, evo_stream_t stream) {
+    if (Bt < 0 || N < 0 || C < 0 || workspace_bytes < 0 || (outgoing != 0 && outgoing != 1))
+        return EVO_ERR_INVALID_ARG;
+    if (dtype != EVO_DTYPE_BF16 && dtype != EVO_DTYPE_FP16)
+        return EVO_ERR_UNSUPPORTED_DTYPE;
+    if (Bt == 0 || N == 0 || C == 0) return EVO_OK;
+    if (!A || !Bm || !Z || !workspace) return EVO_ERR_INVALID_ARG;
+    int64_t section, total, elems, bytes;
+    if (!trimul_layout(Bt, N, C, &section, &total) || !mul_ok(Bt, N, &elems) || !mul_ok(elems, N, &elems) ||
+        !mul_ok(elems, C, &elems) || !mul_ok(elems, 2, &bytes))
+        return EVO_ERR_UNSUPPORTED_SHAPE;
+    if (workspace_bytes < total) return EVO_ERR_INVALID_ARG;
+    const int64_t int_max = 2147483647, tiles_mn = (N + 127) / 128;
+    int64_t tiles;
+    if (N > int_max || C > int_max || Bt * N > int_max || (N + 31) / 32 > 65535 || (C + 31) / 32 > 65535 ||
+        !mul_ok(Bt * C, tiles_mn * tiles_mn, &tiles) || tiles > int_max || Bt * C > int_max)
+        return EVO_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(A, 2) || !aligned(Bm, 2) || !aligned(Z, 2)) return EVO_ERR_MISALIGNED;
+    if (!aligned(workspace, 256)) return EVO_ERR_MISALIGNED;
+    if (overlap(Z, bytes, A, bytes) || overlap(Z, bytes, Bm, bytes) || overlap(workspace, total, A, bytes) ||
+        overlap(workspace, total, Bm, bytes) || overlap(workspace, total, Z, bytes))
+        return EVO_ERR_INVALID_ARG;
+    RelaxedCapture relaxed;
+    DeviceScope scope;
+    const int dev = select_device_of(A, scope);
+    if (dev < 0) return dev;
+    if (dev >= kMaxDevices) return EVO_ERR_UNSUPPORTED_SHAPE;
+    for (const void* ptr : {Bm, static_cast<const void*>(Z), static_cast<const void*>(workspace)})
+        if (device_of(ptr) != dev) return EVO_ERR_INVALID_ARG;
+    if (encode_fn() == nullptr) return EVO_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const bool f16 = dtype == EVO_DTYPE_FP16;
+    if (outgoing)
+        return f16 ? launch_trimul<true, true>(dev, A, Bm, Z, workspace, Bt, N, C, st)
+                   : launch_trimul<true, false>(dev, A, Bm, Z, workspace, Bt, N, C, st);
+    return f16 ? launch_trimul<false, true>(dev, A, Bm, Z, workspace, Bt, N, C, st)
+               : launch_trimul<false, false>(dev, A, Bm, Z, workspace, Bt, N, C, st);
 }

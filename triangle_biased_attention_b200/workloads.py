@@ -260,3 +260,21 @@ def sample_slices(case_or_shape, count: int, seed: int, must_include_n=()) -> li
             seen.add(t)
             chosen.append(t)
     return chosen
+
+
+# Triangle multiplication: A, B [Bt, N, N, C] edge representations, standard
+# normal draws (A then B) from PCG64(seed), rounded to the dtype.  Named
+# sizes: the pair representation of an N-residue crop with the usual 128
+# channels.
+TRIMUL_WORKLOADS = {
+    "trimul_768": (1, 768, 128),
+    "trimul_1024": (1, 1024, 128),
+}
+
+
+def trimul_case(Bt: int, N: int, C: int, dtype: torch.dtype, seed: int):
+    """(A, B) host tensors for the triangle multiplication."""
+    rng = _rng(seed)
+    a = _normal(rng, (Bt, N, N, C))
+    b = _normal(rng, (Bt, N, N, C))
+    return _to(a, dtype), _to(b, dtype)
