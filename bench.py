@@ -52,6 +52,11 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="tri_1024", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--op", default="attn", choices=["attn", "trimul"],
+                    help="attn: biased attention (--pass fwd|bwd); trimul: the triangle-multiplication "
+                         "contraction on --trimul-workload")
+    ap.add_argument("--trimul-workload", default="trimul_768", choices=sorted(W.TRIMUL_WORKLOADS))
+    ap.add_argument("--incoming", action="store_true", help="trimul: the incoming direction")
     ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
                     help="fwd: the forward pass (the headline metric); bwd: the backward pass "
                          "(evo_attn_bwd: dQ, dK, dV and the requested bias gradients)")
@@ -539,12 +544,93 @@ def run_ours_bwd(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def run_ours_trimul(args, rank, world, local):
+    """Triangle multiplication: each step is one evo_trimul call (two transposes
+    to channel-first copies, the tcgen05 batched GEMM, the transpose back)."""
+    import triangle_biased_attention_b200 as evo
+    Bt, N, C = W.TRIMUL_WORKLOADS[args.trimul_workload]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    a_h, b_h = W.trimul_case(Bt, N, C, torch.bfloat16, args.seed + rank)
+    a, b = a_h.to(dev), b_h.to(dev)
+    z = torch.empty_like(a)
+    ws = torch.empty(evo.evo_trimul_workspace_size(Bt, N, C), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(dev)
+    outgoing = not args.incoming
+
+    def step():
+        evo.trimul(a, b, outgoing, out=z, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    if evo.evo_attn_sync_status(stream.cuda_stream) != evo.EVO_OK:
+        raise RuntimeError("kernel status")
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with sampler:
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for _ in range(args.steps):
+                step()
+            stop.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = start.elapsed_time(stop)
+    if evo.evo_attn_sync_status(stream.cuda_stream) != evo.EVO_OK:
+        raise RuntimeError("kernel status")
+    ms_max = max_over_ranks(ms, world, dev)
+    flops = 2 * Bt * C * N ** 3
+    alg = 3 * Bt * N * N * C * 2
+    value = world * flops * args.steps / (ms_max * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms / args.steps * 1e-3) / 1e12
+    t_flop = flops / (peaks["bf16_tflops"] * 1e12)
+    t_mem = alg / (peaks["hbm_gbs"] * 1e9)
+    roof = {"bound": "tensor" if t_flop >= t_mem else "hbm", "achieved": achieved, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+            "peak_source": f"{peak_src} (MEASURED_PEAKS.json burst figure)" if peak_src == "measured"
+            else "fallback (6.65 TB/s, 1.59 PFLOP/s)",
+            "alg_flops_per_launch": flops, "alg_bytes_per_launch": alg,
+            "timed": "whole evo_trimul call (two transposes in, the GEMM, one transpose out)"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle.trimul as OT
+        import time as _t
+        # the oracle on a bounded sample: a few channels of the same problem
+        cs = max(1, min(C, 8))
+        t0 = _t.perf_counter()
+        OT.trimul(a_h[..., :cs], b_h[..., :cs], outgoing)
+        sec = _t.perf_counter() - t0
+        cpu = {"value": 2 * Bt * cs * N ** 3 / sec / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+               "kind": "oracle", "cpu": cpu_model(), "nproc": os.cpu_count(),
+               "sample": f"{cs} of {C} channels of {args.trimul_workload} ({sec:.1f} s, float64 numpy matmul)"}
+    if rank == 0:
+        line = {
+            "metric": "triangle multiplication TFLOP/s (2*Bt*C*N^3 flops)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded numpy PCG64, bf16)",
+            "config": {"workload": args.trimul_workload, "Bt": Bt, "N": N, "C": C,
+                       "direction": "outgoing" if outgoing else "incoming",
+                       "l2": "inputs (%.2f GB) larger than the 126 MB L2; no flush" % (alg / 1e9),
+                       "parallelism": "replicas (one full workload per GPU)"},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": None, "gpu_launches": 4 * args.steps,
+            "kernel": "evo_trimul_gemm_kernel", "clocks": sampler.record(),
+        }
+        print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     rank, world, local = dist_setup(args)
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.op == "trimul":
+            run_ours_trimul(args, rank, world, local)
         elif args.which == "bwd":
             run_ours_bwd(args, rank, world, local)
         else:

@@ -1002,14 +1002,17 @@ int launch_trimul(int dev, const void* A, const void* Bm, void* Z, void* workspa
     T* bc = reinterpret_cast<T*>(ws + section);
     T* zc = reinterpret_cast<T*>(ws + 2 * section);
 
+    // 16-byte transposes when every row is whole 16-byte units, else 2-byte ones
+    const bool vec = Cc % 8 == 0 && aligned(A, 16) && aligned(Bm, 16) && aligned(Z, 16);
+    const int tw = vec ? 64 : 32;
+    auto to_cfirst = vec ? evo::evo_trimul_to_cfirst_v<T> : evo::evo_trimul_to_cfirst<T>;
+    auto to_clast = vec ? evo::evo_trimul_to_clast_v<T> : evo::evo_trimul_to_clast<T>;
     cudaLaunchConfig_t cfg = {};
     cfg.stream = st;
     cfg.blockDim = dim3(256, 1, 1);
-    cfg.gridDim = dim3(unsigned(Bt * N), unsigned((N + 31) / 32), unsigned((Cc + 31) / 32));
-    if (cudaLaunchKernelEx(&cfg, evo::evo_trimul_to_cfirst<T>, static_cast<const T*>(A), ac, int(N), int(Cc),
-                           int(np)) != cudaSuccess ||
-        cudaLaunchKernelEx(&cfg, evo::evo_trimul_to_cfirst<T>, static_cast<const T*>(Bm), bc, int(N), int(Cc),
-                           int(np)) != cudaSuccess)
+    cfg.gridDim = dim3(unsigned(Bt * N), unsigned((N + tw - 1) / tw), unsigned((Cc + tw - 1) / tw));
+    if (cudaLaunchKernelEx(&cfg, to_cfirst, static_cast<const T*>(A), ac, int(N), int(Cc), int(np)) != cudaSuccess ||
+        cudaLaunchKernelEx(&cfg, to_cfirst, static_cast<const T*>(Bm), bc, int(N), int(Cc), int(np)) != cudaSuccess)
         return EVO_ERR_CUDA;
 
     // the channel matrices as a 3-D tensor {N (columns), N (rows), Bt*C}, rows
@@ -1040,8 +1043,8 @@ int launch_trimul(int dev, const void* A, const void* Bm, void* Z, void* workspa
     gc.gridDim = dim3(unsigned(p.num_tiles < sms ? p.num_tiles : sms), 1, 1);
     gc.dynamicSmemBytes = Cfg::SMEM_BYTES;
     if (cudaLaunchKernelEx(&gc, kernel, ta, tb, p) != cudaSuccess) return EVO_ERR_CUDA;
-    return cudaLaunchKernelEx(&cfg, evo::evo_trimul_to_clast<T>, static_cast<const T*>(zc), static_cast<T*>(Z),
-                              int(N), int(Cc), int(np)) == cudaSuccess
+    return cudaLaunchKernelEx(&cfg, to_clast, static_cast<const T*>(zc), static_cast<T*>(Z), int(N), int(Cc),
+                              int(np)) == cudaSuccess
                ? EVO_OK
                : EVO_ERR_CUDA;
 }

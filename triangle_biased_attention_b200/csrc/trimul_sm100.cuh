@@ -82,6 +82,91 @@ __global__ void __launch_bounds__(256) evo_trimul_to_clast(const T* __restrict__
     }
 }
 
+// The same two transposes with 16-byte global accesses, for C a multiple of 8
+// and 16-byte aligned pointers: a block moves a 64 x 64 tile (rows of 8
+// 16-byte vectors on both sides) through shared memory; 256 threads, 2
+// vectors each.
+// Writes of the channel-first copies may run into the row padding (columns
+// N .. ldq - 1), which is never read.
+// Element (row, col) of a 64 x 64 16-bit tile in shared memory: rows of 128 B,
+// the 16-byte vector index XORed with bits 3-5 of the row, so that a column
+// read by 8 threads 8 rows apart falls in 8 different banks.
+__device__ __forceinline__ int tr_idx(int row, int col) {
+    return row * 64 + ((((col >> 3) ^ (row >> 3)) & 7) << 3) + (col & 7);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) evo_trimul_to_cfirst_v(const T* __restrict__ x, T* __restrict__ y, int N,
+                                                              int C, int ldq) {
+    __shared__ __align__(16) uint16_t tile[64 * 64];  // [q][c]
+    const int q0 = blockIdx.y * 64, c0 = blockIdx.z * 64;
+    const long long bp = blockIdx.x;
+    const long long b = bp / N;
+    const int p = int(bp - b * N);
+    const uint16_t* xs = reinterpret_cast<const uint16_t*>(x);
+    uint16_t* ys = reinterpret_cast<uint16_t*>(y);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int v = threadIdx.x + 256 * h;  // 64 rows (q) x 8 vectors (c)
+        const int r = v >> 3, cv = (v & 7) * 8;
+        const int q = q0 + r, c = c0 + cv;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (q < N && c < C) val = *reinterpret_cast<const uint4*>(xs + (size_t(bp) * N + q) * C + c);
+        *reinterpret_cast<uint4*>(&tile[tr_idx(r, cv)]) = val;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int v = threadIdx.x + 256 * h;  // 64 rows (c) x 8 vectors (q)
+        const int r = v >> 3, qv = (v & 7) * 8;
+        const int c = c0 + r, q = q0 + qv;
+        if (c < C && q < ldq) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                w[e] = uint32_t(tile[tr_idx(qv + 2 * e, r)]) | (uint32_t(tile[tr_idx(qv + 2 * e + 1, r)]) << 16);
+            *reinterpret_cast<uint4*>(ys + ((size_t(b) * C + c) * N + p) * size_t(ldq) + q) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) evo_trimul_to_clast_v(const T* __restrict__ y, T* __restrict__ z, int N,
+                                                             int C, int ldj) {
+    __shared__ __align__(16) uint16_t tile[64 * 64];  // [c][j]
+    const int j0 = blockIdx.y * 64, c0 = blockIdx.z * 64;
+    const long long bi = blockIdx.x;
+    const long long b = bi / N;
+    const int i = int(bi - b * N);
+    const uint16_t* ys = reinterpret_cast<const uint16_t*>(y);
+    uint16_t* zs = reinterpret_cast<uint16_t*>(z);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int v = threadIdx.x + 256 * h;  // 64 rows (c) x 8 vectors (j)
+        const int r = v >> 3, jv = (v & 7) * 8;
+        const int c = c0 + r, j = j0 + jv;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (c < C && j < ldj)
+            val = *reinterpret_cast<const uint4*>(ys + ((size_t(b) * C + c) * N + i) * size_t(ldj) + j);
+        *reinterpret_cast<uint4*>(&tile[tr_idx(r, jv)]) = val;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int v = threadIdx.x + 256 * h;  // 64 rows (j) x 8 vectors (c)
+        const int r = v >> 3, cv = (v & 7) * 8;
+        const int j = j0 + r, c = c0 + cv;
+        if (j < N && c < C) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                w[e] = uint32_t(tile[tr_idx(cv + 2 * e, r)]) | (uint32_t(tile[tr_idx(cv + 2 * e + 1, r)]) << 16);
+            *reinterpret_cast<uint4*>(zs + (size_t(bi) * N + j) * C + c) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
 // --------------------------------------------------------------- batched GEMM
 
 struct TrimulParams {
