@@ -1034,8 +1034,9 @@ int launch_trimul(int dev, const void* A, const void* Bm, void* Z, void* workspa
     p.zc = reinterpret_cast<uint16_t*>(zc);
     p.N = int(N);
     p.ldz = int(np);
-    p.tiles_mn = int((N + 127) / 128);
-    p.num_tiles = int(Bt * Cc * p.tiles_mn * p.tiles_mn);
+    p.tiles_m = int((N + 127) / 128);
+    p.tiles_n = int((N + Cfg::BN - 1) / Cfg::BN);
+    p.num_tiles = int(Bt * Cc * p.tiles_m * p.tiles_n);
     p.k_steps = int((N + 63) / 64);
     cudaLaunchConfig_t gc = {};
     gc.stream = st;

@@ -16,7 +16,7 @@
 //  * a tiled transpose to channel-first [Bt*C, N, Np] (Np = N rounded up to
 //    8, so that every row is a whole number of 16-byte units for TMA);
 //  * a persistent tcgen05 batched GEMM over the (b, c) channel matrices,
-//    128 x 128 output tiles, K in steps of 64 through a 4-stage TMA ring, the
+//    128 x 256 output tiles, K in steps of 64 through a 4-stage TMA ring, the
 //    fp32 accumulator double-buffered in tensor memory so that a tile's
 //    epilogue overlaps the next tile's MMAs.  Outgoing reads both operands
 //    K-major (k contiguous: rows of the channel-first copies); incoming reads
@@ -172,27 +172,34 @@ __global__ void __launch_bounds__(256) evo_trimul_to_clast_v(const T* __restrict
 struct TrimulParams {
     uint16_t* zc;    // [Bt*C, N, ldz] channel-first result (bf16 / fp16 bits)
     int N, ldz;
-    int tiles_mn;    // ceil(N / 128)
-    int num_tiles;   // Bt * C * tiles_mn^2
+    int tiles_m;     // ceil(N / 128): row blocks
+    int tiles_n;     // ceil(N / BN): column blocks
+    int num_tiles;   // Bt * C * tiles_m * tiles_n
     int k_steps;     // ceil(N / 64)
 };
 
+// Output tiles of 128 rows x BN = 256 columns: one M = 128, N = 256 MMA per
+// 16-deep K step (an MMA instruction costs about the same time at N = 256 as
+// at N = 128, so the wider tile halves the instructions per flop).
 template <bool OUTGOING, bool F16>
 struct TrimulCfg {
     static constexpr int THREADS = 256;  // warp 0 loads, warp 1 MMAs, warps 4-7 epilogue
+    static constexpr int BN = 256;
     static constexpr int STAGES = 4;
-    static constexpr int OPER = 128 * 128;             // one operand stage: 128 x 64 bf16 = 16 KB
-    static constexpr int STAGE_BYTES = 2 * OPER;
+    static constexpr int OPER = 128 * 128;             // A stage: 128 rows x 64 k of bf16 = 16 KB
+    static constexpr int OPER_B = BN * 128;            // B stage: BN x 64 k = 32 KB
+    static constexpr int STAGE_BYTES = OPER + OPER_B;
     static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
     static constexpr int BAR_FULL = 0, BAR_EMPTY = STAGES, BAR_AF = 2 * STAGES, BAR_AE = 2 * STAGES + 2,
                          BAR_DRAIN = 2 * STAGES + 4, NUM_BARS = 2 * STAGES + 5;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-    static constexpr uint32_t TMEM_COLS = 256;         // two 128-column accumulators
+    static constexpr uint32_t TMEM_COLS = 2 * BN;      // two BN-column accumulators
     static constexpr uint32_t AB = F16 ? 0u : ((1u << 7) | (1u << 10));
     static constexpr uint32_t MAJ = OUTGOING ? 0u : ((1u << 15) | (1u << 16));
-    static constexpr uint32_t IDESC = (1u << 4) | AB | MAJ | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+    static constexpr uint32_t IDESC =
+        (1u << 4) | AB | MAJ | ((uint32_t(BN) >> 3) << 17) | ((128u >> 4) << 24);
 };
 
 template <bool OUTGOING, bool F16>
@@ -211,10 +218,10 @@ evo_trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
     // tile L: column block fastest, then row block, then channel matrix
     auto tile = [&](int L, int& tj, int& ti, int& bc) {
-        tj = L % p.tiles_mn;
-        const int r = L / p.tiles_mn;
-        ti = r % p.tiles_mn;
-        bc = r / p.tiles_mn;
+        tj = L % p.tiles_n;
+        const int r = L / p.tiles_n;
+        ti = r % p.tiles_m;
+        bc = r / p.tiles_m;
     };
 
     if (threadIdx.x == 0) {
@@ -258,18 +265,17 @@ evo_trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                     const uint32_t a = sb + uint32_t(s * C::STAGE_BYTES), b = a + C::OPER;
                     const uint32_t f = bar(C::BAR_FULL + s);
                     ptx::mbar_arrive_expect_tx(f, C::STAGE_BYTES);
-                    if (OUTGOING) {
-                        // rows i (resp. j) of the channel matrix, 64 k per row; two 64-row boxes
-                        ptx::tma_load_3d(a, &tm_a, f, 64 * kt, 128 * ti, bc);
-                        ptx::tma_load_3d(a + C::OPER / 2, &tm_a, f, 64 * kt, 128 * ti + 64, bc);
-                        ptx::tma_load_3d(b, &tm_b, f, 64 * kt, 128 * tj, bc);
-                        ptx::tma_load_3d(b + C::OPER / 2, &tm_b, f, 64 * kt, 128 * tj + 64, bc);
-                    } else {
-                        // rows k, 64 i (resp. j) per row; two boxes cover the 128-wide tile
-                        ptx::tma_load_3d(a, &tm_a, f, 128 * ti, 64 * kt, bc);
-                        ptx::tma_load_3d(a + C::OPER / 2, &tm_a, f, 128 * ti + 64, 64 * kt, bc);
-                        ptx::tma_load_3d(b, &tm_b, f, 128 * tj, 64 * kt, bc);
-                        ptx::tma_load_3d(b + C::OPER / 2, &tm_b, f, 128 * tj + 64, 64 * kt, bc);
+                    // 64 x 64 boxes: outgoing, rows i (resp. j) of 64 k each; incoming,
+                    // rows k of 64 i (resp. j) each
+#pragma unroll
+                    for (int x = 0; x < 2; ++x) {
+                        if (OUTGOING) ptx::tma_load_3d(a + 8192 * x, &tm_a, f, 64 * kt, 128 * ti + 64 * x, bc);
+                        else ptx::tma_load_3d(a + 8192 * x, &tm_a, f, 128 * ti + 64 * x, 64 * kt, bc);
+                    }
+#pragma unroll
+                    for (int x = 0; x < C::BN / 64; ++x) {
+                        if (OUTGOING) ptx::tma_load_3d(b + 8192 * x, &tm_b, f, 64 * kt, C::BN * tj + 64 * x, bc);
+                        else ptx::tma_load_3d(b + 8192 * x, &tm_b, f, C::BN * tj + 64 * x, 64 * kt, bc);
                     }
                 }
                 __syncwarp();
@@ -294,7 +300,7 @@ evo_trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
             ok = wait_warp(bar(C::BAR_AE + acc), ((t >> 1) & 1) ^ 1, abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-            const uint32_t d = tmem + uint32_t(128 * acc);
+            const uint32_t d = tmem + uint32_t(C::BN * acc);
             for (int kt = 0; kt < p.k_steps; ++kt, ++n) {
                 const int s = n % C::STAGES;
                 ok = wait_warp(bar(C::BAR_FULL + s), uint32_t(n / C::STAGES) & 1u, abort_flag);
@@ -309,9 +315,9 @@ evo_trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
                         da = desc_k_major<128>(a + 32 * kk);
                         db = desc_k_major<128>(b + 32 * kk);
                     } else {
-                        // MN-major: rows are k (128 B of i or j each), two 64-wide atoms 8 KB apart
-                        da = desc_mn_major<128>(a + 2048 * kk, C::OPER / 2);
-                        db = desc_mn_major<128>(b + 2048 * kk, C::OPER / 2);
+                        // MN-major: rows are k (128 B of i or j each), 64-wide atoms 8 KB apart
+                        da = desc_mn_major<128>(a + 2048 * kk, 8192);
+                        db = desc_mn_major<128>(b + 2048 * kk, 8192);
                     }
                     ptx::mma_ss_elect(d, da, db, C::IDESC, (kt > 0 || kk > 0) ? 1u : 0u);
                 }
@@ -343,18 +349,18 @@ evo_trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_co
             const int i = 128 * ti + r;
             uint16_t* row = p.zc + (size_t(bc) * p.N + i) * size_t(p.ldz);
 #pragma unroll 1
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int c4 = 0; c4 < C::BN / 32; ++c4) {
                 float v[32];
-                ptx::tmem_ld_x32(tl + uint32_t(128 * acc + 32 * c4), reinterpret_cast<uint32_t*>(v));
+                ptx::tmem_ld_x32(tl + uint32_t(C::BN * acc + 32 * c4), reinterpret_cast<uint32_t*>(v));
                 ptx::tmem_ld_wait_x32(reinterpret_cast<uint32_t*>(v));
-                if (c4 == 3) {
+                if (c4 == C::BN / 32 - 1) {
                     ptx::tc_fence_before();
                     ptx::mbar_arrive_elect(bar(C::BAR_AE + acc));
                 }
                 if (i < p.N) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int j = 128 * tj + 32 * c4 + 8 * e;
+                        const int j = C::BN * tj + 32 * c4 + 8 * e;
                         if (j < p.ldz) {
                             uint4 o;
                             if constexpr (F16) {

@@ -269,6 +269,7 @@ def sample_slices(case_or_shape, count: int, seed: int, must_include_n=()) -> li
 TRIMUL_WORKLOADS = {
     "trimul_768": (1, 768, 128),
     "trimul_1024": (1, 1024, 128),
+    "trimul_512": (1, 512, 128),   # profiling size (inputs 2 x 67 MB, still larger than L2 together)
 }
 
 
