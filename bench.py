@@ -42,6 +42,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 KERNEL_SOURCES = ["common.cuh", "ptx_sm100.cuh", "tile_sm100.cuh", "fwd_tri_sm100.cuh", "evo_attn.cu"]
 KERNEL_SOURCES_BWD = ["common.cuh", "ptx_sm100.cuh", "tile_sm100.cuh", "bwd_simt.cuh", "bwd_tri_sm100.cuh",
                       "evo_attn.cu"]
+KERNEL_SOURCES_TRIMUL = ["common.cuh", "ptx_sm100.cuh", "tile_sm100.cuh", "trimul_sm100.cuh", "evo_attn.cu"]
 KERNEL_NAME = "evo_fwd_tri_kernel"
 
 
@@ -595,18 +596,25 @@ def run_ours_trimul(args, rank, world, local):
             else "fallback (6.65 TB/s, 1.59 PFLOP/s)",
             "alg_flops_per_launch": flops, "alg_bytes_per_launch": alg,
             "timed": "whole evo_trimul call (two transposes in, the GEMM, one transpose out)"}
+    roof["traffic"] = recorded_traffic("trimul:" + args.trimul_workload, KERNEL_SOURCES_TRIMUL)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle.trimul as OT
-        import time as _t
-        # the oracle on a bounded sample: a few channels of the same problem
-        cs = max(1, min(C, 8))
-        t0 = _t.perf_counter()
-        OT.trimul(a_h[..., :cs], b_h[..., :cs], outgoing)
-        sec = _t.perf_counter() - t0
-        cpu = {"value": 2 * Bt * cs * N ** 3 / sec / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(),
+        # the oracle on a bounded sample of the same problem: channels in
+        # groups of 8 until about 10 s have been spent
+        sec, done = 0.0, 0
+        while sec < 10.0 and done < C:
+            cs = min(8, C - done)
+            t0 = time.perf_counter()
+            OT.trimul(a_h[..., done:done + cs], b_h[..., done:done + cs], outgoing)
+            sec += time.perf_counter() - t0
+            done += cs
+        import numpy as _np
+        cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+        cpu = {"value": 2 * Bt * done * N ** 3 / sec / 1e12, "unit": "TFLOP/s", "cores": cores,
                "kind": "oracle", "cpu": cpu_model(), "nproc": os.cpu_count(),
-               "sample": f"{cs} of {C} channels of {args.trimul_workload} ({sec:.1f} s, float64 numpy matmul)"}
+               "sample": f"{done} of {C} channels of {args.trimul_workload} ({sec:.1f} s, float64 numpy matmul, "
+                         f"numpy {_np.__version__})"}
     if rank == 0:
         line = {
             "metric": "triangle multiplication TFLOP/s (2*Bt*C*N^3 flops)",
