@@ -36,10 +36,12 @@
 // carries one more box holding 1 in its first column (the ones column of
 // dK_aug).  P and dT tiles are two 64-key atoms of 128 B rows (128 B
 // swizzle): K-major for dQ (keys along K), MN-major for dV and dK (keys along
-// M).  Warp roles (384 threads): warp 0 loads, warp 1 issues the MMAs (one
-// elected lane of the converged warp), warps 4-7 compute P and dT (a thread
-// owns one query row), warps 8-11 drain dQ, dK, dV and the dmask column out
-// of tensor memory.  Every wait is bounded; on expiry the CTA records
+// M).  Warp roles: warp 0 loads, warp 1 issues the MMAs (one elected lane of
+// the converged warp); one (D = 64) or two (D <= 32) softmax warpgroups
+// compute P and dT (a thread owns one query row; with two groups, each takes
+// 64 of its 128 keys, so the step's P and dT are written in half the time);
+// the last warpgroup drains dQ, dK, dV and the dmask column out of tensor
+// memory.  Every wait is bounded; on expiry the CTA records
 // EVO_ERR_TIMEOUT, lets its own copies and MMAs finish, frees tensor memory and
 // exits.
 #pragma once
@@ -73,16 +75,26 @@ struct BwdTriParams {
 template <int D, bool HAS_PAIR, bool F16>
 struct BwdCfg {
     static_assert(D == 16 || D == 32 || D == 64, "head dim");
-    static constexpr int THREADS = 384;
+    // softmax warpgroups: 2 at D <= 32, each taking 64 of a row's 128 keys (so
+    // that a step's P and dT are written twice as fast), 1 at D = 64 (whose
+    // epilogue needs more registers than the split leaves)
+    static constexpr int GROUPS = D <= 32 ? 2 : 1;
+    static constexpr int THREADS = 128 * (2 + GROUPS);
+    static constexpr int EPI0 = 4 + 4 * GROUPS;  // first epilogue warp
+    static constexpr int LOW_REGS = 80, HIGH_REGS = 144;  // setmaxnreg split at GROUPS = 2
+    static_assert(GROUPS == 1 || 128 * LOW_REGS + 3 * 128 * HIGH_REGS <= 65536, "register split");
     static constexpr int BOX = kBM * 32;         // 128 rows x 16 columns, 32 B swizzle
     static constexpr int NBOX = D / 16;
     static constexpr int TILE = NBOX * BOX;      // one Q, K, V or dO tile
     static constexpr int QAUG = TILE + BOX;      // Q tile + the ones box
     static constexpr int KV_STAGES = D <= 32 ? 2 : 1;
     static constexpr int Q_STAGES = 2;
-    static constexpr int PAIR_STAGES = HAS_PAIR ? (D <= 32 ? 2 : 1) : 0;
-    static constexpr int PAIR_RING = HAS_PAIR ? PAIR_STAGES : 1;
-    static constexpr int PAIR_BYTES = kBM * kBN * 2;  // two 128 x 64 boxes, 128 B swizzle
+    // pair-bias tiles as a ring of half tiles (128 query rows x 64 keys, 128 B
+    // swizzle): a step uses two, halves 2g and 2g + 1, each read by the
+    // softmax warps of its keys
+    static constexpr int PAIR_SLOTS = HAS_PAIR ? (GROUPS == 2 ? 3 : (D <= 32 ? 4 : 2)) : 0;
+    static constexpr int PAIR_RING = HAS_PAIR ? PAIR_SLOTS : 1;
+    static constexpr int HALF_BYTES = kBM * 64 * 2;
     static constexpr int PT_ATOM = kBM * 128;          // 64 keys x 128 rows
     static constexpr int PT_BYTES = 2 * PT_ATOM;       // P or dT tile
     // shared-memory map (every tile 1024-aligned)
@@ -91,7 +103,7 @@ struct BwdCfg {
     static constexpr int OFF_Q = OFF_V + KV_STAGES * TILE;
     static constexpr int OFF_DO = OFF_Q + Q_STAGES * QAUG;
     static constexpr int OFF_PAIR = OFF_DO + Q_STAGES * TILE;
-    static constexpr int OFF_P = OFF_PAIR + PAIR_STAGES * PAIR_BYTES;
+    static constexpr int OFF_P = OFF_PAIR + PAIR_SLOTS * HALF_BYTES;
     static constexpr int OFF_DT = OFF_P + PT_BYTES;
     static constexpr int OFF_MASK = OFF_DT + PT_BYTES;  // [2][128] f32: (mask - c) log2(e) per key
     // per softmax warp: 32 rows x 32 fp32 of dT (128 B rows, 128 B swizzle),
@@ -101,14 +113,14 @@ struct BwdCfg {
     // per dQ warp: 32 rows x 16 fp32 of dQ (64 B rows, 64 B swizzle), added to
     // the fp32 dQ sums by TMA tile reductions, 16 columns at a time
     static constexpr int QSTG_WARP = 32 * 64;
-    static constexpr int OFF_QSTG = OFF_STG + (HAS_PAIR ? 4 * STG_WARP : 0);
+    static constexpr int OFF_QSTG = OFF_STG + (HAS_PAIR ? 4 * GROUPS * STG_WARP : 0);
     static constexpr int OFF_BAR = OFF_QSTG + 4 * QSTG_WARP;
     static constexpr int BAR_KVF = 0;                            // [KV_STAGES] K, V landed
     static constexpr int BAR_KVE = BAR_KVF + KV_STAGES;          // [KV_STAGES] last MMA of the unit done
     static constexpr int BAR_QF = BAR_KVE + KV_STAGES;           // [2] Q, dO landed
     static constexpr int BAR_QE = BAR_QF + Q_STAGES;             // [2] MMAs reading them done
-    static constexpr int BAR_BF = BAR_QE + Q_STAGES;             // [PAIR_RING] bias tile landed
-    static constexpr int BAR_BE = BAR_BF + PAIR_RING;            // [PAIR_RING] read by 4 softmax warps
+    static constexpr int BAR_BF = BAR_QE + Q_STAGES;             // [PAIR_RING] bias half tile landed
+    static constexpr int BAR_BE = BAR_BF + PAIR_RING;            // [PAIR_RING] read by its 4 softmax warps
     static constexpr int BAR_SF = BAR_BE + PAIR_RING;            // S, dP in tensor memory
     static constexpr int BAR_SE = BAR_SF + 1;                    // S, dP read
     static constexpr int BAR_PF = BAR_SE + 1;                    // P, dT tiles written
@@ -213,8 +225,8 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             ptx::mbar_init(bar(C::BAR_BE + s), 4);
         }
         ptx::mbar_init(bar(C::BAR_SF), 1);
-        ptx::mbar_init(bar(C::BAR_SE), 4);
-        ptx::mbar_init(bar(C::BAR_PF), 4);
+        ptx::mbar_init(bar(C::BAR_SE), 4 * C::GROUPS);
+        ptx::mbar_init(bar(C::BAR_PF), 4 * C::GROUPS);
         ptx::mbar_init(bar(C::BAR_PE), 1);
         ptx::mbar_init(bar(C::BAR_DQF), 1);
         ptx::mbar_init(bar(C::BAR_DQE), 4);
@@ -245,9 +257,12 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     bool aborted = false;
-
+    // With two softmax groups the loader / MMA warpgroup hands registers to the
+    // softmax and epilogue warps (inside each role's branch, so that the
+    // compiler sees which budget each piece of code runs under).
     if (warp == 0) {
         // ------------------------------------------------------------ loads
+        if constexpr (C::GROUPS == 2) ptx::setmaxnreg_dec<C::LOW_REGS>();
         if (lane == 0) {
             ptx::prefetch_tmap(&tm_q);
             ptx::prefetch_tmap(&tm_k);
@@ -291,19 +306,21 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     ptx::tma_load_4d_more_elect(dd + x * C::BOX, &tm_do, bar(C::BAR_QF + st), 16 * x, t.h, s0, bn);
                 ++n_q;
                 if constexpr (HAS_PAIR) {
-                    const int ps = n_b % C::PAIR_RING;
-                    ok = wait_warp(bar(C::BAR_BE + ps), ((n_b / C::PAIR_RING) & 1) ^ 1, abort_flag);
-                    if (!ok) break;
-                    if (lane == 0) {
-                        const uint32_t dst = sb + C::OFF_PAIR + uint32_t(ps * C::PAIR_BYTES);
-                        const int bh = t.b * p.H + t.h;
-                        ptx::mbar_arrive_expect_tx(bar(C::BAR_BF + ps), C::PAIR_BYTES);
-                        ptx::tma_load_3d(dst, &tm_pair, bar(C::BAR_BF + ps), t.kb * kBN, s0, bh);
-                        ptx::tma_load_3d(dst + C::PAIR_BYTES / 2, &tm_pair, bar(C::BAR_BF + ps), t.kb * kBN + 64, s0,
-                                         bh);
+                    // the step's two half tiles (keys 0-63, 64-127), each in its ring slot
+                    for (int x = 0; x < 2 && ok; ++x) {
+                        const int ps = n_b % C::PAIR_RING;
+                        ok = wait_warp(bar(C::BAR_BE + ps), ((n_b / C::PAIR_RING) & 1) ^ 1, abort_flag);
+                        if (!ok) break;
+                        if (lane == 0) {
+                            const uint32_t dst = sb + C::OFF_PAIR + uint32_t(ps * C::HALF_BYTES);
+                            ptx::mbar_arrive_expect_tx(bar(C::BAR_BF + ps), C::HALF_BYTES);
+                            ptx::tma_load_3d(dst, &tm_pair, bar(C::BAR_BF + ps), t.kb * kBN + 64 * x, s0,
+                                             t.b * p.H + t.h);
+                        }
+                        __syncwarp();
+                        ++n_b;
                     }
-                    __syncwarp();
-                    ++n_b;
+                    if (!ok) break;
                 }
             }
         }
@@ -327,6 +344,7 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMAs
+        if constexpr (C::GROUPS == 2) ptx::setmaxnreg_dec<C::LOW_REGS>();
         struct Step {
             bool valid;
             int g, qb, kvs, uc;
@@ -420,9 +438,16 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             wait_bounded(bar(C::BAR_DRAIN), 0, nullptr);
             __syncwarp();
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp < 4) {
+        if constexpr (C::GROUPS == 2) ptx::setmaxnreg_dec<C::LOW_REGS>();
+    } else if (warp < C::EPI0) {
         // --------------------------------------------------- P and dT rows
-        const int wq = warp - 4;
+        if constexpr (C::GROUPS == 2) ptx::setmaxnreg_inc<C::HIGH_REGS>();
+        // group grp takes the 32-key chunks c0 .. c1 - 1 of every row
+        const int grp = (warp - 4) >> 2;
+        const int sw = warp - 4;                      // stage of this warp's dpair tiles
+        const int c0 = grp * (4 / C::GROUPS), c1 = c0 + 4 / C::GROUPS;
+        const int wq = (warp - 4) & 3;
         const int r = 32 * wq + lane;                 // query row in the block; key index for the mask row
         const uint32_t tl = tmem + (uint32_t(32 * wq) << 16);
         float* mask_w = reinterpret_cast<float*>(smem + C::OFF_MASK);
@@ -444,7 +469,7 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int j = t.kb * kBN + r;
             mbits = 0u;
             c = 0.f;
-            if (p.mask != nullptr && j < p.S) {
+            if (grp == 0 && p.mask != nullptr && j < p.S) {
                 mbits = p.mask[size_t(t.bn) * p.S + j];
                 c = __ldg(p.cmask + t.bn);
             }
@@ -473,9 +498,12 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     const float x = (p.mask != nullptr) ? bits_to_f32<F16>(mbits) - cm : 0.f;
                     ml = (x < -kMaskFloor) ? -INFINITY : x * kLog2e;
                 }
-                mask_w[mb * kBN + r] = ml;
-                __syncwarp();
-                ptx::mbar_arrive_elect(bar(C::BAR_MKF + mb));
+                // the first group writes the row, every group waits for it
+                if (grp == 0) {
+                    mask_w[mb * kBN + r] = ml;
+                    __syncwarp();
+                    ptx::mbar_arrive_elect(bar(C::BAR_MKF + mb));
+                }
                 ok = wait_warp(bar(C::BAR_MKF + mb), uint32_t(uc >> 1) & 1u, abort_flag);
                 if (!ok) break;
             }
@@ -488,20 +516,21 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (!ok) break;
                 ptx::tc_fence_after();
                 const float lse2 = (lr == INFINITY) ? INFINITY : lr * kLog2e;
-                const int ps = HAS_PAIR ? g % C::PAIR_RING : 0;
-                if constexpr (HAS_PAIR) {
-                    ok = wait_warp(bar(C::BAR_BF + ps), uint32_t(g / C::PAIR_RING) & 1u, abort_flag);
-                    if (!ok) break;
-                }
-                const uint32_t ptile = sb + C::OFF_PAIR + uint32_t(ps * C::PAIR_BYTES);
+                // this step's pair-bias half tiles are numbers 2g (keys 0-63) and 2g + 1 of the ring
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = c0; c < c1; ++c) {
+                    const int hs = (2 * g + (c >> 1)) % C::PAIR_RING;
+                    if (HAS_PAIR && (c & 1) == 0) {
+                        ok = wait_warp(bar(C::BAR_BF + hs), uint32_t((2 * g + (c >> 1)) / C::PAIR_RING) & 1u,
+                                       abort_flag);
+                        if (!ok) break;
+                    }
                     float s[32], dp[32];
                     ptx::tmem_ld_x32(tl + C::TM_S + 32u * c, reinterpret_cast<uint32_t*>(s));
                     ptx::tmem_ld_x32(tl + C::TM_DP + 32u * c, reinterpret_cast<uint32_t*>(dp));
                     ptx::tmem_ld_wait_x32(reinterpret_cast<uint32_t*>(s));
                     ptx::reg_fence_x32(reinterpret_cast<uint32_t*>(dp));
-                    if (c == 3) {
+                    if (c == c1 - 1) {
                         ptx::tc_fence_before();
                         ptx::mbar_arrive_elect(bar(C::BAR_SE));
                     }
@@ -515,7 +544,7 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         s[4 * q4 + 3] = fmaf(s[4 * q4 + 3], p.scale_log2, m4.w - lse2);
                     }
                     if constexpr (HAS_PAIR) {
-                        const uint32_t base = ptile + uint32_t((c / 2) * (C::PAIR_BYTES / 2));
+                        const uint32_t base = sb + C::OFF_PAIR + uint32_t(hs * C::HALF_BYTES);
 #pragma unroll
                         for (int u4 = 0; u4 < 4; ++u4) {
                             const uint4 w = ptx::ld_shared_v4(base + swz_chunk<128>(r, (c % 2) * 4 + u4));
@@ -538,7 +567,7 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         pw[e / 2] = pack2<F16>(s[e], s[e + 1]);
                         dw[e / 2] = pack2<F16>(dp[e], dp[e + 1]);
                     }
-                    if (c == 0 && g > 0) {
+                    if (c == c0 && g > 0) {
                         // the MMAs of the previous step have read the P and dT tiles
                         ok = wait_warp(bar(C::BAR_PE), uint32_t(g - 1) & 1u, abort_flag);
                         if (!ok) break;
@@ -557,7 +586,7 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         // added to dpair by one TMA tile reduction (whole 128 B rows in L2);
                         // lane 0 issues it and first waits until the previous one has
                         // read the stage
-                        const uint32_t stg = sb + C::OFF_STG + uint32_t(wq * C::STG_WARP);
+                        const uint32_t stg = sb + C::OFF_STG + uint32_t(sw * C::STG_WARP);
                         if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
                         __syncwarp();
 #pragma unroll
@@ -576,12 +605,13 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                         }
                     }
+                    if (HAS_PAIR && (c & 1) == 1) {
+                        // the last chunk of this half tile has read it
+                        __syncwarp();
+                        ptx::mbar_arrive_elect(bar(C::BAR_BE + hs));
+                    }
                 }
                 if (!ok) break;
-                if constexpr (HAS_PAIR) {
-                    __syncwarp();
-                    ptx::mbar_arrive_elect(bar(C::BAR_BE + ps));
-                }
                 ptx::fence_proxy_async_smem();  // generic-proxy writes -> tensor-core reads
                 __syncwarp();
                 ptx::mbar_arrive_elect(bar(C::BAR_PF));
@@ -591,9 +621,10 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
         __syncwarp();
         if (!ok) aborted = true;
-    } else if (warp >= 8) {
+    } else {
         // ------------------------------------------- dQ, dK, dV, dmask out
-        const int we = warp - 8;
+        if constexpr (C::GROUPS == 2) ptx::setmaxnreg_inc<C::HIGH_REGS>();
+        const int we = warp - C::EPI0;
         const int r = 32 * we + lane;
         const uint32_t tl = tmem + (uint32_t(32 * we) << 16);
         constexpr int LDW = D >= 32 ? 32 : 16;  // columns per tensor-memory load

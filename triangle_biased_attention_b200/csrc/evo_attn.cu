@@ -752,6 +752,13 @@ int launch_bwd_tri(int dev, const void* Q, const void* K, const void* V, const v
     auto kernel = evo::evo_bwd_tri_kernel<D, HAS_PAIR, F16>;
     static AttrOnce attr;
     if (!attr.ensure(dev, kernel, C::SMEM_BYTES)) return EVO_ERR_CUDA;
+    if (C::GROUPS == 2) {
+        // the register hand-over (setmaxnreg) needs the whole split at launch
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess ||
+            fa.numRegs * C::THREADS < 128 * C::LOW_REGS + 3 * 128 * C::HIGH_REGS)
+            return EVO_ERR_CUDA;
+    }
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
         return EVO_ERR_CUDA;
