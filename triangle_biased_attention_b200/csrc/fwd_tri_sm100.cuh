@@ -36,13 +36,14 @@
 //    numbers per key that sum exactly to the fp32 (mask - c) * sqrt(D), c the
 //    running mask maximum of the slice; keys past S get -inf).
 //  * Softmax in base 2, 32 keys per step: t = S + pair * sqrt(D) (packed fp32
-//    FMA), the step maximum, p = 2^(t log2(e) / sqrt(D) - m) against the
-//    running maximum m, P packed to fp16 and stored, the row sum accumulated in
-//    registers.  m only moves when a step exceeds it by more than 15 (p stays
-//    <= 2^15, inside fp16; the result is exact after the division by the row
-//    sum).  When it does, the P already stored for the block and the O
-//    accumulator are rescaled in tensor memory.  The first step of a tile
-//    always sets m this way.
+//    FMA), p = 2^(t log2(e) / sqrt(D) - m) against the running maximum m, P
+//    packed to fp16 and stored, the row sum accumulated in registers.  m only
+//    moves when a step exceeds it by more than 15 (p stays <= 2^15, inside
+//    fp16; the result is exact after the division by the row sum).  The step's
+//    p sum tells: at most 2^15, no p of the step is above it, so the step
+//    maximum is only formed when the sum is larger.  When m moves, the P
+//    already stored for the block and the O accumulator are rescaled in
+//    tensor memory.  The first step of a tile always sets m this way.
 //  * Every wait is bounded (about two seconds); on expiry the CTA records
 //    EVO_ERR_TIMEOUT, drains its own in-flight copies and MMAs, frees tensor
 //    memory and exits.
@@ -79,6 +80,9 @@ struct TriParams {
 // The running maximum moves when a step exceeds it by more than this (log2
 // units): p <= 2^15 keeps P inside fp16 (largest finite 65504).
 constexpr float kTriRescaleThreshold = 15.0f;
+// A step's p sum above this (2^kTriRescaleThreshold) may hold a p past the
+// threshold; at or below it none does.
+constexpr float kStepSumLimit = 32768.0f;
 
 // Slices per tile: as many as tensor memory holds, each a 128-column score
 // buffer plus a D-column O accumulator.
@@ -92,7 +96,7 @@ struct TriCfg {
     // register split (setmaxnreg) where the launch leaves less than the
     // softmax needs: the helper warpgroup hands registers to the softmax
     static constexpr bool SPLIT_REGS = NS >= 2;
-    static constexpr int HELPER_REGS = NS == 3 ? 80 : 96;
+    static constexpr int HELPER_REGS = NS == 3 ? 72 : 96;
     static constexpr int SOFTMAX_REGS = NS == 3 ? 144 : 200;
     static_assert(!SPLIT_REGS || 128 * HELPER_REGS + NS * 128 * SOFTMAX_REGS <= THREADS * (65536 / THREADS / 8 * 8),
                   "register split");
@@ -284,12 +288,10 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    if constexpr (C::SPLIT_REGS) {
-        if (warp < 4) ptx::setmaxnreg_dec<C::HELPER_REGS>();
-        else ptx::setmaxnreg_inc<C::SOFTMAX_REGS>();
-    }
-
+    // The register hand-over (setmaxnreg) sits at the top of each role's
+    // branch, so that the compiler sees which budget the role's code runs under.
     if (warp < 4) {
+        if constexpr (C::SPLIT_REGS) ptx::setmaxnreg_dec<C::HELPER_REGS>();
         if (warp == 0) {
             // ------------------------------------------ bias tiles and masks
             // The bias tile of every (tile, block), shared by the three
@@ -639,6 +641,7 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
     } else {
         // ------------------------------------------------------------ softmax
+        if constexpr (C::SPLIT_REGS) ptx::setmaxnreg_inc<C::SOFTMAX_REGS>();
         const int w = (warp - 4) >> 2;   // slice (n0 + w)
         const int quarter = warp & 3;    // TMEM lanes 32*quarter .. +31
         const int r = quarter * 32 + lane;
@@ -766,13 +769,12 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     if (!kEarlyS) tmem_ld_x32f(tS + 32u * c, s);
                     load_bias(c, bw);
                     tmem_wait_x32f(s);
-                    // One basic block per step: t = S + pair * sqrt(D), the step
-                    // maximum, and p = 2^(t log2(e) / sqrt(D) - m) against the
-                    // current m, all independent per key pair, so the exp unit
-                    // is fed while the adds and maxima proceed.  The check that
-                    // m still covers the step comes after; when it does not
-                    // (rare), the step is recomputed from t (kept in s).
-                    float mx0 = -INFINITY, mx1 = -INFINITY;
+                    // One basic block per step: t = S + pair * sqrt(D) and
+                    // p = 2^(t log2(e) / sqrt(D) - m) against the current m, all
+                    // independent per key pair, so the exp unit is fed while the
+                    // adds proceed.  The check that m still covers the step comes
+                    // after; when it does not (rare), the step is recomputed from
+                    // t (kept in s).
                     float2 csa = make_float2(0.f, 0.f), csb = make_float2(0.f, 0.f);
                     uint32_t pk[16];
                     {
@@ -785,8 +787,6 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             else tt = make_float2(s[k], s[k + 1]);
                             s[k] = tt.x;
                             s[k + 1] = tt.y;
-                            if (e & 1) mx1 = max3f(mx1, tt.x, tt.y);
-                            else mx0 = max3f(mx0, tt.x, tt.y);
                             const float2 x = __ffma2_rn(tt, sc2, nm2);
                             const float p0 = ptx::ex2_approx(x.x);
                             const float p1 = ptx::ex2_approx(x.y);
@@ -810,11 +810,18 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             for (int e = 0; e < 16; ++e) step_pair(e, 0.f, 0.f);
                         }
                     }
-                    const float mx = fmaxf(mx0, mx1);
-                    const bool raise = mx > thr;
-                    if (__any_sync(0xffffffffu, raise)) {
-                        // The step exceeds the running maximum by more than 15
-                        // (always so for the first step of a tile): move m to
+                    // The step's p sum bounds each of its p: at most 2^15 means
+                    // every p fits (the maximum is only needed when it does not,
+                    // and at the first step of a tile, where m is still -inf).
+                    const float2 cst = __fadd2_rn(csa, csb);
+                    const bool check = (cst.x + cst.y > kStepSumLimit) || (m == -INFINITY);
+                    if (__any_sync(0xffffffffu, check)) {
+                        float mx = -INFINITY;
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) mx = max3f(mx, s[e], s[e + 1]);
+                        const bool raise = mx > thr;
+                        // Where the step exceeds the running maximum by more than
+                        // 15 (always so for the first step of a tile): move m to
                         // the step maximum, rescale what is already accumulated
                         // relative to the old m, and recompute this step.
                         float alpha = 1.f;
