@@ -199,6 +199,19 @@ __device__ __forceinline__ float2 pair_to_f32x2(uint32_t w) {
         return make_float2(ptx::bf16lo_to_f32(w), ptx::bf16hi_to_f32(w));
     }
 }
+// t = b * q + s for the two bf16 numbers of one 32-bit word (low half first),
+// packed fp32: the word's halves become the fp32 pair in place (a shift and a
+// mask) and feed one packed FMA.
+__device__ __forceinline__ float2 bf16x2_fma2(uint32_t w, float2 q, float2 s) {
+    unsigned long long d;
+    asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 bb, ss, qq;\n\t"
+        "shl.b32 lo, %1, 16;\n\tand.b32 hi, %1, 0xffff0000;\n\t"
+        "mov.b64 bb, {lo, hi};\n\tmov.b64 ss, {%2, %3};\n\tmov.b64 qq, {%4, %5};\n\t"
+        "fma.rn.f32x2 %0, bb, qq, ss;\n\t}"
+        : "=l"(d)
+        : "r"(w), "f"(s.x), "f"(s.y), "f"(q.x), "f"(q.y));
+    return make_float2(__uint_as_float(uint32_t(d)), __uint_as_float(uint32_t(d >> 32)));
+}
 // Two fp32 -> the output type, round to nearest even; `lo` in the low half.
 template <bool F16>
 __device__ __forceinline__ uint32_t pack_out(float lo, float hi) {
@@ -780,11 +793,13 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     {
                         const float m_safe = (m == -INFINITY) ? 0.f : m;  // an all -inf row keeps p = 0
                         const float2 nm2 = make_float2(-m_safe, -m_safe);
-                        auto step_pair = [&](int e, float b0, float b1) {
+                        auto step_pair = [&](int e, uint32_t bwd) {
                             const int k = 2 * e;
                             float2 tt;
-                            if (HAS_PAIR) tt = __ffma2_rn(make_float2(b0, b1), sqd2, make_float2(s[k], s[k + 1]));
-                            else tt = make_float2(s[k], s[k + 1]);
+                            const float2 sv = make_float2(s[k], s[k + 1]);
+                            if (!HAS_PAIR) tt = sv;
+                            else if constexpr (F16) tt = __ffma2_rn(pair_to_f32x2<F16>(bwd), sqd2, sv);
+                            else tt = bf16x2_fma2(bwd, sqd2, sv);
                             s[k] = tt.x;
                             s[k + 1] = tt.y;
                             const float2 x = __ffma2_rn(tt, sc2, nm2);
@@ -800,14 +815,13 @@ evo_fwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                 const uint32_t wd[4] = {bw[q].x, bw[q].y, bw[q].z, bw[q].w};
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
-                                    const float2 b = pair_to_f32x2<F16>(wd[e]);
-                                    step_pair(4 * q + e, b.x, b.y);
+                                    step_pair(4 * q + e, wd[e]);
                                 }
                             }
                             if (bias_tma && c == 3) ptx::mbar_arrive_elect(bar(C::BAR_BE + bs));
                         } else {
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) step_pair(e, 0.f, 0.f);
+                            for (int e = 0; e < 16; ++e) step_pair(e, 0u);
                         }
                     }
                     // The step's p sum bounds each of its p: at most 2^15 means
