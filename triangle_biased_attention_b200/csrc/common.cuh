@@ -59,9 +59,10 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
     }
 }
 
-// Inline fast path: one try_wait, then the bounded slow path.
+// Inline fast path: one non-blocking test (cheaper than a try_wait when the
+// phase has already completed, the common case), then the bounded slow path.
 __device__ __forceinline__ bool wait_fast(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (ptx::mbar_test_wait(bar, parity)) return true;
     return wait_bounded(bar, parity, abort_flag);
 }
 
