@@ -42,9 +42,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                  : "memory");
 }
 
-// True once the phase with the given parity has completed.  The thread may
-// be suspended until the phase completes or `suspend_ns` has passed, so a
-// waiting warp takes no issue slots from the warps that do the work.
 // Non-blocking test of a phase: returns at once, whether or not it completed.
 __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
@@ -58,6 +55,9 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// True once the phase with the given parity has completed.  The thread may
+// be suspended until the phase completes or `suspend_ns` has passed, so a
+// waiting warp takes no issue slots from the warps that do the work.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uint32_t suspend_ns = 1000000u) {
     uint32_t ok;
     asm volatile(
