@@ -517,13 +517,15 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ptx::tc_fence_after();
                 const float lse2 = (lr == INFINITY) ? INFINITY : lr * kLog2e;
                 // this step's pair-bias half tiles are numbers 2g (keys 0-63) and 2g + 1 of the ring
-#pragma unroll 1
-                for (int c = c0; c < c1; ++c) {
+                // One 32-key chunk: P and dT packed into pw, dw, its dT tile added to
+                // dpair (the reduction needs no wait for the previous step's MMAs, so
+                // it is issued before the P and dT stores)
+                auto chunk = [&](int c, uint32_t* pw, uint32_t* dw) -> bool {
                     const int hs = (2 * g + (c >> 1)) % C::PAIR_RING;
                     if (HAS_PAIR && (c & 1) == 0) {
                         ok = wait_warp(bar(C::BAR_BF + hs), uint32_t((2 * g + (c >> 1)) / C::PAIR_RING) & 1u,
                                        abort_flag);
-                        if (!ok) break;
+                        if (!ok) return false;
                     }
                     float s[32], dp[32];
                     ptx::tmem_ld_x32(tl + C::TM_S + 32u * c, reinterpret_cast<uint32_t*>(s));
@@ -557,7 +559,6 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             }
                         }
                     }
-                    uint32_t pw[16], dw[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
                         s[e] = ptx::ex2_approx(s[e]);
@@ -566,20 +567,6 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         dp[e + 1] = s[e + 1] * (dp[e + 1] - dl);
                         pw[e / 2] = pack2<F16>(s[e], s[e + 1]);
                         dw[e / 2] = pack2<F16>(dp[e], dp[e + 1]);
-                    }
-                    if (c == c0 && g > 0) {
-                        // the MMAs of the previous step have read the P and dT tiles
-                        ok = wait_warp(bar(C::BAR_PE), uint32_t(g - 1) & 1u, abort_flag);
-                        if (!ok) break;
-                    }
-                    const uint32_t poff = uint32_t((c / 2) * C::PT_ATOM);
-#pragma unroll
-                    for (int u4 = 0; u4 < 4; ++u4) {
-                        const uint32_t off = poff + swz_chunk<128>(r, (c % 2) * 4 + u4);
-                        ptx::st_shared_v4(sb + C::OFF_P + off,
-                                          make_uint4(pw[4 * u4], pw[4 * u4 + 1], pw[4 * u4 + 2], pw[4 * u4 + 3]));
-                        ptx::st_shared_v4(sb + C::OFF_DT + off,
-                                          make_uint4(dw[4 * u4], dw[4 * u4 + 1], dw[4 * u4 + 2], dw[4 * u4 + 3]));
                     }
                     if (HAS_PAIR && p.dpair_acc != nullptr) {
                         // this warp's 32 rows x 32 keys of dT, staged in shared memory and
@@ -609,6 +596,40 @@ evo_bwd_tri_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         // the last chunk of this half tile has read it
                         __syncwarp();
                         ptx::mbar_arrive_elect(bar(C::BAR_BE + hs));
+                    }
+                    return true;
+                };
+                auto store = [&](int c, const uint32_t* pw, const uint32_t* dw) {
+                    const uint32_t poff = uint32_t((c / 2) * C::PT_ATOM);
+#pragma unroll
+                    for (int u4 = 0; u4 < 4; ++u4) {
+                        const uint32_t off = poff + swz_chunk<128>(r, (c % 2) * 4 + u4);
+                        ptx::st_shared_v4(sb + C::OFF_P + off,
+                                          make_uint4(pw[4 * u4], pw[4 * u4 + 1], pw[4 * u4 + 2], pw[4 * u4 + 3]));
+                        ptx::st_shared_v4(sb + C::OFF_DT + off,
+                                          make_uint4(dw[4 * u4], dw[4 * u4 + 1], dw[4 * u4 + 2], dw[4 * u4 + 3]));
+                    }
+                };
+                if constexpr (C::GROUPS == 2) {
+                    // both chunks first (they overlap the previous step's MMAs), then
+                    // the wait for those MMAs to have read the P and dT tiles
+                    uint32_t pwa[16], dwa[16], pwb[16], dwb[16];
+                    ok = chunk(c0, pwa, dwa) && chunk(c0 + 1, pwb, dwb);
+                    if (ok && g > 0) ok = wait_warp(bar(C::BAR_PE), uint32_t(g - 1) & 1u, abort_flag);
+                    if (!ok) break;
+                    store(c0, pwa, dwa);
+                    store(c0 + 1, pwb, dwb);
+                } else {
+#pragma unroll 1
+                    for (int c = c0; c < c1; ++c) {
+                        uint32_t pw[16], dw[16];
+                        if (!(ok = chunk(c, pw, dw))) break;
+                        if (c == c0 && g > 0) {
+                            // the MMAs of the previous step have read the P and dT tiles
+                            ok = wait_warp(bar(C::BAR_PE), uint32_t(g - 1) & 1u, abort_flag);
+                            if (!ok) break;
+                        }
+                        store(c, pw, dw);
                     }
                 }
                 if (!ok) break;
