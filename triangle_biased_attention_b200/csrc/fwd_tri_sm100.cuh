@@ -96,8 +96,8 @@ struct TriCfg {
     // register split (setmaxnreg) where the launch leaves less than the
     // softmax needs: the helper warpgroup hands registers to the softmax
     static constexpr bool SPLIT_REGS = NS >= 2;
-    static constexpr int HELPER_REGS = NS == 3 ? 72 : 96;
-    static constexpr int SOFTMAX_REGS = NS == 3 ? 144 : 200;
+    static constexpr int HELPER_REGS = NS == 3 ? 72 : 136;
+    static constexpr int SOFTMAX_REGS = NS == 3 ? 144 : 176;
     static_assert(!SPLIT_REGS || 128 * HELPER_REGS + NS * 128 * SOFTMAX_REGS <= THREADS * (65536 / THREADS / 8 * 8),
                   "register split");
     // a Q/K/V row is D bf16; rows wider than 128 B are split into sub-tiles of
