@@ -154,6 +154,13 @@ int launch_tri(int dev, const void* Q, const void* K, const void* V, const void*
     const CUtensorMapDataType dt = F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     static AttrOnce attr;
     if (!attr.ensure(dev, kernel, C::SMEM_BYTES)) return EVO_ERR_CUDA;
+    if (C::SPLIT_REGS) {
+        // the register hand-over (setmaxnreg) needs the whole split at launch
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess ||
+            fa.numRegs * C::THREADS < 128 * C::HELPER_REGS + C::NS * 128 * C::SOFTMAX_REGS)
+            return EVO_ERR_CUDA;
+    }
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
         return EVO_ERR_CUDA;
