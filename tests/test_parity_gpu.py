@@ -2,6 +2,8 @@
 the same seeded inputs.  Small shapes are compared element by element; the
 full-size workloads are compared on every element where the oracle finishes
 in seconds and on sampled (b, n, h) slices otherwise."""
+import dataclasses
+
 import pytest
 import torch
 
@@ -110,6 +112,30 @@ def test_bf16_late_maximum_raises(shape):
     B, N, S, H, D, mask, spike, frac, seed = shape
     case = W.random_case(B, N, S, H, D, torch.bfloat16, seed=seed, mask=mask, pair=True,
                          spike_frac=frac, spike=spike)
+    check_full(case, str(shape))
+
+
+# Pair bias rising by a fixed amount every 32 keys (one softmax step of the
+# tensor-core kernel): with +6 per step (8.7 in log2 units) each new step's p
+# reach 2^8.7 against the running maximum, so the step's p sum passes 2^15
+# while no single p does (the check's rare path without a raise); with +12
+# (17.3 in log2 units) every step raises the maximum and rescales P and O.
+RAMP_SHAPES = [
+    # B, N, S, H, D, ramp per 32 keys, seed
+    (1, 3, 256, 2, 32, 6.0, 31),
+    (1, 3, 384, 1, 32, 12.0, 32),
+    (1, 2, 200, 2, 64, 6.0, 33),
+    (1, 3, 160, 1, 16, 12.0, 34),
+]
+
+
+@pytest.mark.parametrize("shape", RAMP_SHAPES, ids=lambda s: f"S{s[2]}-D{s[4]}-ramp{s[5]:g}")
+def test_bf16_rising_steps(shape):
+    B, N, S, H, D, ramp, seed = shape
+    case = W.random_case(B, N, S, H, D, torch.bfloat16, seed=seed, mask="none", pair=True)
+    steps = (torch.arange(S) // 32).to(torch.float32) * ramp           # per key
+    pair = (case.pair.float() + steps.view(1, 1, 1, 1, S)).to(torch.bfloat16)
+    case = dataclasses.replace(case, pair=pair)
     check_full(case, str(shape))
 
 
